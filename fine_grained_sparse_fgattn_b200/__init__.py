@@ -1,0 +1,154 @@
+"""Tile-sparse softmax attention (FG-Attn style) on NVIDIA B200, sm_100a.
+
+A thin ctypes binding over the C ABI in include/fgattn.h.  Every step of the
+computation runs in the library's CUDA kernels; this module only checks
+tensors, passes their device pointers and the current CUDA stream, and turns
+status codes into exceptions.  PyTorch supplies device memory and streams.
+There is no CPU path: if libfgattn.so cannot be loaded, importing this package
+fails.
+
+Method: "FG-Attn: Leveraging Fine-Grained Sparse Attention in Video Diffusion
+Models", Abstract -- score computations are skipped for whole M x N tiles
+(M >= 16 queries, N >= 1 keys); skipped scores count as -inf.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+from . import _build
+
+__all__ = ["kept_capacity", "compact_mask", "forward", "device_error", "status_string", "num_sms",
+           "FgattnError", "LIB_PATH", "DEVERR_BAD_INDEX", "DEVERR_BAD_COUNT", "DEVERR_TIMEOUT"]
+
+LIB_PATH = _build.LIB
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_DEVICE = range(6)
+DEVERR_BAD_INDEX, DEVERR_BAD_COUNT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
+
+
+def _load() -> ctypes.CDLL:
+    if not _build.is_current():
+        try:
+            _build.build()
+        except Exception as e:  # no silent fallback: the CUDA library is the product
+            raise ImportError(f"libfgattn.so is missing or stale and could not be built: {e}") from e
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, p, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+    lib.fgattn_kept_capacity.argtypes = [i64]
+    lib.fgattn_kept_capacity.restype = i64
+    lib.fgattn_compact_mask.argtypes = [p, i64, i64, i64, i64, i64, p, p, i64, p]
+    lib.fgattn_compact_mask.restype = i32
+    lib.fgattn_forward.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float, p, p, p]
+    lib.fgattn_forward.restype = i32
+    lib.fgattn_device_error.argtypes = [p, i32, ctypes.POINTER(ctypes.c_uint32)]
+    lib.fgattn_device_error.restype = i32
+    lib.fgattn_num_sms.argtypes = []
+    lib.fgattn_num_sms.restype = i32
+    lib.fgattn_status_string.argtypes = [i32]
+    lib.fgattn_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+class FgattnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def status_string(status: int) -> str:
+    return _lib.fgattn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise FgattnError(status, where)
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtypes) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def kept_capacity(L: int) -> int:
+    """Per-row stride of kept_idx: L rounded up to 16."""
+    return int(_lib.fgattn_kept_capacity(int(L)))
+
+
+def num_sms() -> int:
+    return int(_lib.fgattn_num_sms())
+
+
+def compact_mask(mask: torch.Tensor, B: int, H: int, L: int, M: int, N: int,
+                 kept_idx: Optional[torch.Tensor] = None, kept_cnt: Optional[torch.Tensor] = None,
+                 cap: Optional[int] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Packed tile mask uint32/int32 [B,H,QB,W] -> (kept_idx int32 [B,H,QB,cap], kept_cnt int32 [B,H,QB])."""
+    QB = -(-L // M)
+    cap = kept_capacity(L) if cap is None else int(cap)
+    dev = mask.device
+    if kept_idx is None:
+        kept_idx = torch.empty((B, H, QB, cap), dtype=torch.int32, device=dev)
+    if kept_cnt is None:
+        kept_cnt = torch.empty((B, H, QB), dtype=torch.int32, device=dev)
+    st = _lib.fgattn_compact_mask(_dev(mask, "mask", (torch.int32, torch.uint32)), B, H, L, M, N,
+                                  _dev(kept_idx, "kept_idx", (torch.int32,)),
+                                  _dev(kept_cnt, "kept_cnt", (torch.int32,)), cap, _stream_ptr(stream))
+    _check(st, "fgattn_compact_mask")
+    return kept_idx, kept_cnt
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kept_idx: Optional[torch.Tensor],
+            kept_cnt: Optional[torch.Tensor], M: int, N: int, scale: Optional[float] = None,
+            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+            stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Tile-sparse attention forward.  q, k, v: bf16 [B,H,L,d].  kept_idx None = dense run.
+
+    Returns (out bf16 [B,H,L,d], lse fp32 [B,H,L] natural-log, or None)."""
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, H, L, d] shape")
+    B, H, L, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    bf = (torch.bfloat16,)
+    qp, kp, vp = _dev(q, "q", bf), _dev(k, "k", bf), _dev(v, "v", bf)
+    op = _dev(out, "out", bf)
+    lp = _dev(lse, "lse", (torch.float32,)) if lse is not None else None
+    if kept_idx is not None:
+        ip = _dev(kept_idx, "kept_idx", (torch.int32,))
+        cp = _dev(kept_cnt, "kept_cnt", (torch.int32,))
+        cap = kept_idx.shape[-1]
+    else:
+        ip = cp = None
+        cap = L
+    st = _lib.fgattn_forward(qp, kp, vp, ip, cp, cap, B, H, L, d, M, N, scale, op, lp, _stream_ptr(stream))
+    _check(st, "fgattn_forward")
+    return out, lse
+
+
+def device_error(clear: bool = True, stream=None) -> int:
+    """Synchronise the stream and return the kernels' device error bits (DEVERR_*)."""
+    bits = ctypes.c_uint32(0)
+    st = _lib.fgattn_device_error(_stream_ptr(stream), 1 if clear else 0, ctypes.byref(bits))
+    if st not in (OK, ERR_DEVICE):
+        _check(st, "fgattn_device_error")
+    return int(bits.value)

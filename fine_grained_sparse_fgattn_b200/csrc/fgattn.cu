@@ -1,0 +1,145 @@
+// C ABI of the tile-sparse attention library (declared in include/fgattn.h).
+// Host side only: argument validation, launch configuration, device error
+// word.  The kernels are in compact_mask.cuh and attention_fwd.cuh.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "fgattn.h"
+#include "attention_fwd.cuh"
+#include "compact_mask.cuh"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return sms;
+}
+
+template <int D, int MQ>
+fgattn_status launch_fwd(const fgattn::FwdParams& prm, cudaStream_t stream) {
+    using C = fgattn::FwdCfg<D, MQ>;
+    // Request enough shared memory that exactly one block is resident per SM:
+    // the grid is persistent (one block per SM, static round-robin over work).
+    const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;
+    static bool configured = false;  // per process; the attribute is per function
+    if (!configured) {
+        if (cudaFuncSetAttribute(fgattn::fgattn_fwd_kernel<D, MQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem) != cudaSuccess)
+            return FGATTN_ERR_CUDA;
+        configured = true;
+    }
+    const int sms = current_sms();
+    if (sms <= 0) return FGATTN_ERR_CUDA;
+    const int64_t grid = prm.items < sms ? prm.items : sms;
+    fgattn::fgattn_fwd_kernel<D, MQ><<<(unsigned)grid, C::THREADS, smem, stream>>>(prm);
+    return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t fgattn_kept_capacity(int64_t L) {
+    if (L < 1) return -1;
+    return (L + 15) / 16 * 16;
+}
+
+fgattn_status fgattn_compact_mask(const uint32_t* mask, int64_t B, int64_t H, int64_t L, int64_t M, int64_t N,
+                                  int32_t* kept_idx, int32_t* kept_cnt, int64_t cap, fgattn_stream_t stream) {
+    if (!mask || !kept_idx || !kept_cnt) return FGATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || L < 1 || M < 1 || N < 1) return FGATTN_ERR_INVALID_ARG;
+    if (L > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
+    if (!aligned16(kept_idx) || (reinterpret_cast<uintptr_t>(mask) & 3u)) return FGATTN_ERR_INVALID_ARG;
+    if (cap < L || (cap & 3)) return FGATTN_ERR_CAPACITY;
+    const int64_t QB = (L + M - 1) / M;
+    const int64_t G = (L + N - 1) / N;
+    const int64_t W = (G + 31) / 32;
+    const int64_t rows = B * H * QB;
+    const int64_t blocks = (rows + 7) / 8;
+    if (blocks > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
+    fgattn::compact_mask_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(mask, rows, QB, L, M, N, G, W,
+                                                                                      kept_idx, kept_cnt, cap);
+    return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
+}
+
+fgattn_status fgattn_forward(const void* q, const void* k, const void* v, const int32_t* kept_idx,
+                             const int32_t* kept_cnt, int64_t cap, int64_t B, int64_t H, int64_t L, int64_t d,
+                             int64_t M, int64_t N, float scale, void* out, float* lse, fgattn_stream_t stream) {
+    if (!q || !k || !v || !out) return FGATTN_ERR_INVALID_ARG;
+    if (kept_idx && !kept_cnt) return FGATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || L < 1 || M < 1 || N < 1 || d < 1) return FGATTN_ERR_INVALID_ARG;
+    if (L > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return FGATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FGATTN_ERR_INVALID_ARG;
+    if (kept_idx && (reinterpret_cast<uintptr_t>(kept_idx) & 3u)) return FGATTN_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FGATTN_ERR_INVALID_ARG;
+    if (kept_idx && cap < L) return FGATTN_ERR_CAPACITY;
+    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
+
+    fgattn::FwdParams prm;
+    prm.q = static_cast<const __nv_bfloat16*>(q);
+    prm.k = static_cast<const __nv_bfloat16*>(k);
+    prm.v = static_cast<const __nv_bfloat16*>(v);
+    prm.kept_idx = kept_idx;
+    prm.kept_cnt = kept_cnt;
+    prm.out = static_cast<__nv_bfloat16*>(out);
+    prm.lse = lse;
+    prm.cap = kept_idx ? cap : L;
+    prm.L = L;
+    prm.QB = (L + M - 1) / M;
+    prm.items = B * H * prm.QB;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    (void)N;  // the key lists already encode the tile width
+
+    cudaStream_t s = (cudaStream_t)stream;
+    if (d == 128) {
+        switch (M) {
+            case 16: return launch_fwd<128, 16>(prm, s);
+            case 32: return launch_fwd<128, 32>(prm, s);
+            case 64: return launch_fwd<128, 64>(prm, s);
+            default: return launch_fwd<128, 128>(prm, s);
+        }
+    }
+    switch (M) {
+        case 16: return launch_fwd<64, 16>(prm, s);
+        case 32: return launch_fwd<64, 32>(prm, s);
+        case 64: return launch_fwd<64, 64>(prm, s);
+        default: return launch_fwd<64, 128>(prm, s);
+    }
+}
+
+fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* bits) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FGATTN_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, fgattn::g_device_error, sizeof(word)) != cudaSuccess) return FGATTN_ERR_CUDA;
+    if (clear && word) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(fgattn::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return FGATTN_ERR_CUDA;
+    }
+    if (bits) *bits = word;
+    return word ? FGATTN_ERR_DEVICE : FGATTN_OK;
+}
+
+int fgattn_num_sms(void) { return current_sms(); }
+
+const char* fgattn_status_string(fgattn_status status) {
+    switch (status) {
+        case FGATTN_OK: return "ok";
+        case FGATTN_ERR_INVALID_ARG: return "invalid argument";
+        case FGATTN_ERR_UNSUPPORTED: return "unsupported head dimension or query-block height";
+        case FGATTN_ERR_CAPACITY: return "kept-index capacity smaller than the sequence length";
+        case FGATTN_ERR_CUDA: return "CUDA runtime or launch error";
+        case FGATTN_ERR_DEVICE: return "a kernel reported a device-side error";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

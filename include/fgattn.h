@@ -1,0 +1,130 @@
+/*
+ * fgattn.h -- C ABI of the B200 (sm_100a) tile-sparse attention library.
+ *
+ * The operation is the forward pass of softmax attention in which whole
+ * M x N score tiles (M queries x N keys, M >= 16, N >= 1) are skipped; a
+ * skipped score contributes exactly as if it were -inf.  Source: "FG-Attn:
+ * Leveraging Fine-Grained Sparse Attention in Video Diffusion Models",
+ * Abstract.  The page fixes neither the mask layout, the interface nor the
+ * precision; this header states the readings the library implements.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library allocates no device memory per call and keeps no reference to
+ *     any pointer after the call returns.
+ *   - Work is enqueued on `stream` (0 = the legacy default stream) and runs
+ *     asynchronously; argument validation happens synchronously on the host
+ *     before anything is enqueued, and a call that returns an error status has
+ *     enqueued nothing.
+ *   - Shapes: B batch, H heads, L tokens, d head dimension.
+ *       QB = ceil(L / M) query blocks, G = ceil(L / N) key groups,
+ *       W  = ceil(G / 32) mask words per query block.
+ *   - Layouts (all contiguous, row-major, innermost last):
+ *       q, k, v, out : bf16   [B][H][L][d]
+ *       lse          : fp32   [B][H][L]         (natural logarithm)
+ *       mask         : uint32 [B][H][QB][W]     tile (qb, g) kept <=> bit (g % 32)
+ *                                               of word g / 32 is 1 (LSB first);
+ *                                               bits >= G are ignored
+ *       kept_idx     : int32  [B][H][QB][cap]   ascending kept key indices
+ *       kept_cnt     : int32  [B][H][QB]        number of valid entries per row
+ *   - Diagonal rule: whatever the mask says, query block qb keeps the key
+ *     groups that hold its own rows' indices, floor(qb*M/N) ..
+ *     floor((min(qb*M+M, L) - 1) / N), so every query row has at least one
+ *     kept key and a finite log-sum-exp.
+ *   - Ragged ends: keys >= L do not exist (the last group has L - (G-1)*N
+ *     keys); query rows >= L are not computed and not written.
+ *   - Pointer alignment: 16 bytes for q, k, v, out, kept_idx.
+ *   - Errors never abort the process; every entry point returns a status.
+ */
+#ifndef FGATTN_H
+#define FGATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fgattn_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    FGATTN_OK = 0,
+    FGATTN_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, misaligned pointer, bad scale */
+    FGATTN_ERR_UNSUPPORTED = 2, /* a legal value this build has no kernel for (d, M) */
+    FGATTN_ERR_CAPACITY = 3,    /* cap < L: a kept list might not fit */
+    FGATTN_ERR_CUDA = 4,        /* a CUDA runtime call or a launch failed */
+    FGATTN_ERR_DEVICE = 5       /* a kernel flagged an error (see fgattn_device_error) */
+} fgattn_status;
+
+/* Device error bits recorded by the kernels (fgattn_device_error). */
+#define FGATTN_DEVERR_BAD_INDEX 0x1u   /* a kept_idx entry was outside [0, L); a safe row was used */
+#define FGATTN_DEVERR_BAD_COUNT 0x2u   /* a kept_cnt entry was outside [0, cap]; it was clamped */
+#define FGATTN_DEVERR_TIMEOUT 0x4u     /* a pipeline wait exceeded its bound; the block exited */
+
+/*
+ * Stride (in int32 elements) to use for one kept_idx row: L rounded up to a
+ * multiple of 16 (keeps every row 64-byte aligned).  Returns -1 if L < 1.
+ */
+int64_t fgattn_kept_capacity(int64_t L);
+
+/*
+ * Mask compaction ("FG-Attn ...", Abstract: the M x N tiles to compute).
+ * For every row (b, h, qb): kept_idx[row][0 .. kept_cnt[row]) = the key
+ * indices of every kept group of the row, after the diagonal rule, ascending;
+ * entries past kept_cnt[row] are left untouched.  Bit-exact integer work.
+ *   mask      in   device uint32 [B][H][QB][W]
+ *   kept_idx  out  device int32  [B][H][QB][cap], cap >= L, cap % 4 == 0
+ *   kept_cnt  out  device int32  [B][H][QB]
+ * Requires 1 <= M, 1 <= N (the method itself asks M >= 16; the compaction
+ * accepts any M >= 1).  Errors: INVALID_ARG, CAPACITY, CUDA.
+ */
+fgattn_status fgattn_compact_mask(const uint32_t* mask, int64_t B, int64_t H, int64_t L, int64_t M,
+                                  int64_t N, int32_t* kept_idx, int32_t* kept_cnt, int64_t cap,
+                                  fgattn_stream_t stream);
+
+/*
+ * Tile-sparse attention forward ("FG-Attn ...", Abstract: scores of skipped
+ * tiles are never computed and count as -inf).  For each query row i of
+ * block qb, over the keys j listed in kept_idx for (b, h, qb):
+ *   s_ij = scale * q_i . k_j,  p_ij = exp(s_ij - m_i),  l_i = sum_j p_ij,
+ *   out_i = sum_j p_ij v_j / l_i  (stored as bf16),  lse_i = m_i + ln l_i.
+ *   q, k, v   in   device bf16 [B][H][L][d]
+ *   kept_idx  in   device int32 [B][H][QB][cap] (as written by fgattn_compact_mask,
+ *                  or any ascending or unordered list of distinct keys < L),
+ *                  or NULL for a dense run of the same kernel (every key kept)
+ *   kept_cnt  in   device int32 [B][H][QB] (ignored when kept_idx is NULL);
+ *                  every count must be >= 1 and <= cap
+ *   out       out  device bf16 [B][H][L][d]
+ *   lse       out  device fp32 [B][H][L], may be NULL
+ * Supported: d in {64, 128}, M in {16, 32, 64, 128}, any N >= 1, any L >= 1.
+ * Accumulation in fp32; P is rounded to bf16 for the P.V product; the sum l
+ * is taken over the fp32 probabilities.
+ * Errors: INVALID_ARG, UNSUPPORTED, CAPACITY, CUDA.  Kernel-side problems
+ * (corrupt indices or counts, a wait that timed out) never fault: they set a
+ * device error bit that fgattn_device_error reports.
+ */
+fgattn_status fgattn_forward(const void* q, const void* k, const void* v, const int32_t* kept_idx,
+                             const int32_t* kept_cnt, int64_t cap, int64_t B, int64_t H, int64_t L,
+                             int64_t d, int64_t M, int64_t N, float scale, void* out, float* lse,
+                             fgattn_stream_t stream);
+
+/*
+ * Synchronise `stream`, then report (and, if clear != 0, reset) the device
+ * error bits (FGATTN_DEVERR_*) recorded on the current device since the last
+ * clear.  *bits may be NULL.  Returns DEVICE if any bit is set, CUDA if the
+ * synchronisation failed, else OK.
+ */
+fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* bits);
+
+/* Number of streaming multiprocessors the forward kernel's persistent grid uses
+ * on the current device (0 on failure). */
+int fgattn_num_sms(void);
+
+/* Static, human-readable name of a status code. */
+const char* fgattn_status_string(fgattn_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FGATTN_H */

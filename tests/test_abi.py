@@ -1,0 +1,114 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before enqueuing anything (no GPU needed).
+
+The rejection cases pass at least one argument that validation refuses, so no
+kernel is ever launched; they are skipped on a machine with a GPU anyway.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import fine_grained_sparse_fgattn_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fgattn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fgattn_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["fgattn_compact_mask", "fgattn_forward", "fgattn_kept_capacity", "fgattn_status_string",
+              "fgattn_device_error", "fgattn_num_sms"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(F.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} not exported"
+
+
+def test_kept_capacity():
+    assert F.kept_capacity(1) == 16
+    assert F.kept_capacity(16) == 16
+    assert F.kept_capacity(32760) == 32768
+    assert F.kept_capacity(118800) == 118800
+    assert F.kept_capacity(0) == -1
+
+
+def test_status_strings():
+    for s in range(6):
+        assert isinstance(F.status_string(s), str) and F.status_string(s)
+    assert F.status_string(99) == "unknown status"
+
+
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="host-validation cases only run without a GPU")
+
+P = 1 << 20  # a 16-byte-aligned stand-in address; every case below is refused before use
+
+
+def _fwd(**kw):
+    a = dict(q=P, k=P, v=P, idx=P, cnt=P, cap=64, B=1, H=1, L=64, d=128, M=64, N=16, scale=0.1, out=P, lse=P)
+    a.update(kw)
+    return F._lib.fgattn_forward(a["q"], a["k"], a["v"], a["idx"], a["cnt"], a["cap"], a["B"], a["H"], a["L"],
+                                 a["d"], a["M"], a["N"], a["scale"], a["out"], a["lse"], None)
+
+
+def _cmp(**kw):
+    a = dict(mask=P, B=1, H=1, L=64, M=64, N=16, idx=P, cnt=P, cap=64)
+    a.update(kw)
+    return F._lib.fgattn_compact_mask(a["mask"], a["B"], a["H"], a["L"], a["M"], a["N"], a["idx"], a["cnt"],
+                                      a["cap"], None)
+
+
+@no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), F.ERR_INVALID_ARG),
+    (dict(out=None), F.ERR_INVALID_ARG),
+    (dict(cnt=None), F.ERR_INVALID_ARG),
+    (dict(L=0), F.ERR_INVALID_ARG),
+    (dict(B=0), F.ERR_INVALID_ARG),
+    (dict(N=0), F.ERR_INVALID_ARG),
+    (dict(scale=float("nan")), F.ERR_INVALID_ARG),
+    (dict(q=P + 8), F.ERR_INVALID_ARG),
+    (dict(lse=P + 2), F.ERR_INVALID_ARG),
+    (dict(cap=63), F.ERR_CAPACITY),
+    (dict(d=96), F.ERR_UNSUPPORTED),
+    (dict(d=256), F.ERR_UNSUPPORTED),
+    (dict(M=48), F.ERR_UNSUPPORTED),
+    (dict(M=8), F.ERR_UNSUPPORTED),
+    (dict(M=256), F.ERR_UNSUPPORTED),
+])
+def test_forward_rejects(kw, status):
+    assert _fwd(**kw) == status
+
+
+@no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(mask=None), F.ERR_INVALID_ARG),
+    (dict(idx=None), F.ERR_INVALID_ARG),
+    (dict(cnt=None), F.ERR_INVALID_ARG),
+    (dict(L=0), F.ERR_INVALID_ARG),
+    (dict(M=0), F.ERR_INVALID_ARG),
+    (dict(N=0), F.ERR_INVALID_ARG),
+    (dict(H=-1), F.ERR_INVALID_ARG),
+    (dict(idx=P + 4), F.ERR_INVALID_ARG),
+    (dict(cap=48), F.ERR_CAPACITY),
+    (dict(cap=66), F.ERR_CAPACITY),
+])
+def test_compact_rejects(kw, status):
+    assert _cmp(**kw) == status
+
+
+@no_gpu
+def test_valid_call_without_gpu_reports_cuda_error():
+    # All arguments valid, so the launch is attempted; with no device it fails cleanly.
+    assert _cmp() == F.ERR_CUDA
