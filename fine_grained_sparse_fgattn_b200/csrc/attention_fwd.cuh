@@ -1,11 +1,11 @@
-// Tile-sparse softmax attention forward for sm_100a (tcgen05 + TMEM).
+// Tile-sparse softmax attention forward for sm_100a (TMA gather + tcgen05 + TMEM).
 //
 // The method ("FG-Attn: Leveraging Fine-Grained Sparse Attention in Video
 // Diffusion Models", Abstract): score computations are skipped for whole
-// M x N tiles; skipped scores count as -inf.  Here the kept tiles arrive as a
-// per-query-block list of kept key indices (mask compaction), and this kernel
-// gathers only those K/V rows, so the tensor cores always see dense tiles
-// whatever N is.
+// M x N tiles; skipped scores count as -inf.  The kept tiles arrive as a
+// per-query-block list of kept key indices (mask compaction); this kernel
+// gathers only those K/V rows with TMA row gathers, so the tensor cores always
+// see dense 128-key tiles whatever N is.
 //
 // Key-major formulation.  Each work item is one query block (b, h, qb) of MQ
 // rows.  Its kept keys are processed in chunks of 128:
@@ -13,23 +13,29 @@
 //     O^T [D x MQ]        += V_chunk^T [D x 128] . P^T [128 x MQ]  (MMA2, M=D)
 // Putting the gathered keys on the MMA's M dimension keeps every MMA at the
 // full-rate M=128 shape for any query-block height MQ in {16, 32, 64, 128}.
-// A softmax thread owns one key (one TMEM lane) across all MQ queries, so the
-// per-query running maximum is a cross-lane quantity.  It is refreshed lazily:
-// probabilities are taken against a per-query reference mref and only when a
-// score exceeds mref by more than TAU (log2 units) is the reference raised,
-// after which the partial sums and the O accumulator are rescaled.  The final
-// normalisation uses the same reference, so the result is exact up to
-// rounding whatever reference was used.
+// A softmax thread owns one key (TMEM lane) of the chunk; two softmax
+// warpgroups split the chunk's MQ query columns between them.  The per-query
+// running maximum is a cross-lane quantity, so it is refreshed lazily:
+// probabilities are taken against a per-query reference mref, and only when a
+// score exceeds mref by more than TAU (log2 units) is the reference raised and
+// the partial sums and the O accumulator rescaled.  The final normalisation
+// uses the same reference, so the result is exact up to rounding whatever
+// reference was used.
 //
-// Warp roles (256 threads, two warps per SM sub-partition):
-//   warps 0-3  softmax / correction / epilogue (thread t <-> TMEM lane t)
-//   warps 4-6  producer: cp.async gathers of Q, K, V rows into 128B-swizzled
-//              shared memory; completion tracked by mbarriers
-//   warp  7    TMEM allocation + single-thread tcgen05.mma issue
+// Warp roles (512 threads = four warpgroups):
+//   warps 0-3   softmax warpgroup 0: query columns [0, MQ/2)
+//   warps 4-7   softmax warpgroup 1: query columns [MQ/2, MQ)
+//   warps 8-10  K producer: TMA tile load of the query block, TMA gather4 of K rows
+//   warp  11    TMEM allocation + single-thread tcgen05.mma issue
+//   warps 12-15 V producer: cp.async row gathers of V
+// Gathering K and V through the two different copy paths (TMA and the LSU)
+// keeps more row requests in flight per SM than either path alone; the
+// producer warpgroups hand most of their registers to the softmax groups.
 // Every mbarrier wait is bounded; on timeout the block records an error bit,
 // drains its in-flight copies and MMAs, frees TMEM and exits.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include <cstdint>
@@ -45,10 +51,10 @@ constexpr uint32_t kErrBadCount = 0x2u;
 constexpr uint32_t kErrTimeout = 0x4u;
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 
-struct FwdParams {
-    const __nv_bfloat16* q;
-    const __nv_bfloat16* k;
-    const __nv_bfloat16* v;
+struct alignas(64) FwdParams {
+    CUtensorMap tmap_q;  // [B*H*L rows][D], box {64, MQ}, 128B swizzle
+    CUtensorMap tmap_k;  // [B*H*L rows][D], box {64, 1},  128B swizzle (row gathers)
+    const __nv_bfloat16* v_base;  // V rows, gathered with cp.async
     const int32_t* kept_idx;  // nullptr: dense (every key kept)
     const int32_t* kept_cnt;
     __nv_bfloat16* out;
@@ -56,7 +62,7 @@ struct FwdParams {
     int64_t cap;
     int64_t L;
     int64_t QB;
-    int64_t items;  // B * H * QB
+    int64_t items;     // B * H * QB
     float scale_log2;  // scale * log2(e)
 };
 
@@ -64,38 +70,54 @@ template <int D, int MQ>
 struct FwdCfg {
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(MQ == 16 || MQ == 32 || MQ == 64 || MQ == 128, "query block");
-    static constexpr int KC = 128;                      // keys per chunk = MMA1 M
-    static constexpr int NST = (MQ == 128) ? 2 : 3;     // K/V pipeline stages
-    static constexpr int PPR = D / 8;                   // 16-byte pieces per K/V/Q row
-    static constexpr int KV_TILE = KC * D * 2;          // bytes of a K or V chunk
+    static constexpr int KC = 128;              // keys per chunk = MMA1 M
+    static constexpr int CW = MQ / 2;           // query columns per softmax warpgroup
+    static constexpr int KV_TILE = KC * D * 2;  // bytes of a K or V chunk
     static constexpr int P_ROW = (MQ * 2 < 128) ? MQ * 2 : 128;  // bytes per key row of a P panel
-    static constexpr int P_CPR = P_ROW / 16;            // 16-byte chunks per P row
-    static constexpr int P_PANEL = KC * P_ROW;          // bytes per P panel
+    static constexpr int P_CPR = P_ROW / 16;    // 16-byte chunks per P row
+    static constexpr int P_PANEL = KC * P_ROW;  // bytes per P panel
     static constexpr int P_TILE = KC * MQ * 2;
-    static constexpr int KSLOT = (KV_TILE > P_TILE) ? KV_TILE : P_TILE;  // K slot also holds P
     static constexpr int Q_TILE = MQ * D * 2;
-    static constexpr int STAGE_ROWS = 16;               // epilogue staging rows
+    static constexpr int SROWS = (CW < 16) ? CW : 16;  // epilogue staging rows per warpgroup
+    static constexpr int STAGE = SROWS * D * 2;
+    static constexpr int MISC = 2 * (3 * CW + 4 * CW) * 4 + 64 * 8 + 64;  // mref/alpha/lfin/red, barriers
+    static constexpr int LIMIT = 227 * 1024 - 1024 - 256;
+    static constexpr int fixed_bytes(int nk, int nv, int np) {
+        return nk * KV_TILE + nv * KV_TILE + np * P_TILE + Q_TILE + 2 * STAGE + MISC;
+    }
+    // pipeline depths: K ring, V ring, P buffers (deepest that fits)
+    static constexpr int NK = fixed_bytes(3, 2, 1) <= LIMIT ? 3 : 2;
+    static constexpr int NV = fixed_bytes(NK, 3, 2) <= LIMIT ? 3 : 2;
+    static constexpr int NP = fixed_bytes(NK, NV, 2) <= LIMIT ? 2 : 1;
+    static_assert(fixed_bytes(NK, NV, NP) <= LIMIT, "shared memory");
     static constexpr int OFF_K = 0;
-    static constexpr int OFF_V = OFF_K + NST * KSLOT;
-    static constexpr int OFF_Q = OFF_V + NST * KV_TILE;
-    static constexpr int OFF_STAGE = OFF_Q + Q_TILE;
-    static constexpr int OFF_MREF = OFF_STAGE + STAGE_ROWS * D * 2;
-    static constexpr int OFF_ALPHA = OFF_MREF + MQ * 4;
-    static constexpr int OFF_LFIN = OFF_ALPHA + MQ * 4;
-    static constexpr int OFF_RED = OFF_LFIN + MQ * 4;
-    static constexpr int OFF_IDX = OFF_RED + 4 * MQ * 4;   // NST x 128 gathered row indices
-    static constexpr int OFF_BAR = OFF_IDX + NST * KC * 4;
-    // barriers: kv_full[NST], kv_empty[NST], q_full, q_empty, s_full[2], s_free[2],
-    //           p_full[2], o_done[2], drain
-    static constexpr int NBAR = 2 * NST + 11;
+    static constexpr int OFF_V = OFF_K + NK * KV_TILE;
+    static constexpr int OFF_P = OFF_V + NV * KV_TILE;
+    static constexpr int OFF_Q = OFF_P + NP * P_TILE;
+    static constexpr int OFF_STAGE = OFF_Q + Q_TILE;         // 2 x STAGE
+    static constexpr int OFF_MREF = OFF_STAGE + 2 * STAGE;   // [2][CW]
+    static constexpr int OFF_ALPHA = OFF_MREF + 2 * CW * 4;  // [2][CW]
+    static constexpr int OFF_LFIN = OFF_ALPHA + 2 * CW * 4;  // [2][CW]
+    static constexpr int OFF_RED = OFF_LFIN + 2 * CW * 4;    // [2][4][CW]
+    static constexpr int OFF_BAR = (OFF_RED + 2 * 4 * CW * 4 + 7) / 8 * 8;
+    // barriers: k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] q_full q_empty
+    //           s_full[2] s_free[2] p_full[NP] o_done[2] drain
+    static constexpr int B_KFULL = 0, B_KEMPTY = NK, B_VFULL = 2 * NK, B_VEMPTY = 2 * NK + NV;
+    static constexpr int B_QFULL = 2 * NK + 2 * NV, B_QEMPTY = B_QFULL + 1, B_SFULL = B_QFULL + 2;
+    static constexpr int B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_ODONE = B_PFULL + NP;
+    static constexpr int B_DRAIN = B_ODONE + 2, NBAR = B_DRAIN + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
     static constexpr int BYTES = OFF_ABORT + 8;
-    static constexpr int SMEM_REQUEST = BYTES + 1024;    // + alignment slack
+    static_assert(BYTES <= LIMIT, "shared memory layout");
+    static constexpr int SMEM_REQUEST = BYTES + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = (3 * MQ <= 64) ? 64 : (3 * MQ <= 128) ? 128 : (3 * MQ <= 256) ? 256 : 512;
-    static constexpr int THREADS = 256;
-    static constexpr int NPROD = 96;                    // producer threads (warps 4-6)
-    static constexpr bool KEEP = MQ <= 64;              // keep a chunk's scores in registers
+    static constexpr int THREADS = 512;
+    // Register split between the two softmax warpgroups and the two producer/MMA
+    // warpgroups (2*128*SOFT + 2*128*AUX = 512*128).  MQ = 128 keeps 64 columns of
+    // scores and sums per softmax thread and needs the larger share.
+    static constexpr uint32_t SOFT_REGS = MQ == 128 ? 176 : 128;
+    static constexpr uint32_t AUX_REGS = MQ == 128 ? 80 : 128;
 };
 
 // UMMA shared-memory descriptor (sm_100): start, leading/stride byte offsets,
@@ -117,9 +139,9 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn_m
 }
 
 // Byte offset of 16-byte chunk `c` of row `r` in a swizzled panel with `row_bytes`
-// per row (128, 64 or 32): the chunk index is XORed with the row's position in its
-// 8-row swizzle atom, matching both the UMMA canonical layouts and the panel base
-// alignment of 1024 bytes.
+// per row (128, 64 or 32): the chunk index is XORed with the row's position in
+// its 8-row swizzle atom (panel bases are 1024-byte aligned), the layout both
+// the UMMA descriptors and the TMA 128B swizzle use.
 __device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c, uint32_t row_bytes) {
     uint32_t off = r * row_bytes + c * 16u;
     const uint32_t cmask = row_bytes / 16u - 1u;
@@ -157,55 +179,77 @@ __device__ __forceinline__ int64_t item_count(const FwdParams& p, int64_t item, 
     return c;
 }
 
+// Kept-list entries 4*lane .. 4*lane+3 of chunk c (raw, unchecked).  Entries past
+// the list read as 0.  Issued several chunks ahead of use: the lists live in HBM.
+__device__ __forceinline__ int4 fetch_idx(const int32_t* lst, int64_t cnt, int64_t c, int lane) {
+    const int64_t j0 = c * 128 + 4 * lane;
+    if (lst == nullptr) {
+        return make_int4(j0 < cnt ? (int)j0 : 0, j0 + 1 < cnt ? (int)(j0 + 1) : 0, j0 + 2 < cnt ? (int)(j0 + 2) : 0,
+                         j0 + 3 < cnt ? (int)(j0 + 3) : 0);
+    }
+    if (j0 + 3 < cnt) return __ldg(reinterpret_cast<const int4*>(lst + j0));
+    return make_int4(j0 < cnt ? __ldg(lst + j0) : 0, j0 + 1 < cnt ? __ldg(lst + j0 + 1) : 0,
+                     j0 + 2 < cnt ? __ldg(lst + j0 + 2) : 0, j0 + 3 < cnt ? __ldg(lst + j0 + 3) : 0);
+}
+
+// Global row coordinates of four fetched entries.  Entries outside [0, L) are
+// reported and replaced by key 0 of the head (as are entries past the list,
+// whose scores the softmax masks).
+__device__ __forceinline__ void rows_of(const FwdParams& p, int4 raw, int64_t row0, bool report, int32_t (&rows)[4]) {
+    const int32_t idx[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int32_t x = idx[i];
+        if (x < 0 || (int64_t)x >= p.L) {
+            if (report) atomicOr(&g_device_error, kErrBadIndex);
+            x = 0;
+        }
+        rows[i] = (int32_t)(row0 + x);
+    }
+}
+
 template <int D, int MQ>
-__global__ void __launch_bounds__(256, 1) fgattn_fwd_kernel(const FwdParams p) {
+__global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = FwdCfg<D, MQ>;
-    constexpr int NST = C::NST;
+    constexpr int NK = C::NK, NV = C::NV, NP = C::NP, CW = C::CW;
     constexpr float TAU = 8.0f;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
-    float* mref = reinterpret_cast<float*>(smem + C::OFF_MREF);
-    float* alpha = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
-    float* lfin = reinterpret_cast<float*>(smem + C::OFF_LFIN);
-    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
     const uint32_t bar0 = sbase + C::OFF_BAR;
-    auto KV_FULL = [&](int i) { return bar0 + 8u * i; };
-    auto KV_EMPTY = [&](int i) { return bar0 + 8u * (NST + i); };
-    const uint32_t Q_FULL = bar0 + 8u * (2 * NST);
-    const uint32_t Q_EMPTY = bar0 + 8u * (2 * NST + 1);
-    auto S_FULL = [&](int i) { return bar0 + 8u * (2 * NST + 2 + i); };
-    auto S_FREE = [&](int i) { return bar0 + 8u * (2 * NST + 4 + i); };
-    auto P_FULL = [&](int i) { return bar0 + 8u * (2 * NST + 6 + i); };
-    auto O_DONE = [&](int i) { return bar0 + 8u * (2 * NST + 8 + i); };
-    const uint32_t DRAIN = bar0 + 8u * (2 * NST + 10);
-    auto KSLOT = [&](int st) { return sbase + C::OFF_K + (uint32_t)st * C::KSLOT; };
-    auto VSLOT = [&](int st) { return sbase + C::OFF_V + (uint32_t)st * C::KV_TILE; };
+    auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    auto KSLOT = [&](int i) { return sbase + C::OFF_K + (uint32_t)i * C::KV_TILE; };
+    auto VSLOT = [&](int i) { return sbase + C::OFF_V + (uint32_t)i * C::KV_TILE; };
+    auto PBUF = [&](int i) { return sbase + C::OFF_P + (uint32_t)i * C::P_TILE; };
     const uint32_t QTILE = sbase + C::OFF_Q;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    if (warp == 7) {
+    if (warp == 11) {
         ptx::tmem_alloc(sbase + C::OFF_TMEM, C::TMEM_COLS);
         ptx::tmem_relinquish();
     }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NST; ++i) {
-            ptx::mbar_init(KV_FULL(i), C::NPROD);
-            ptx::mbar_init(KV_EMPTY(i), 1);
+        for (int i = 0; i < NK; ++i) {
+            ptx::mbar_init(BAR(C::B_KFULL + i), 3);
+            ptx::mbar_init(BAR(C::B_KEMPTY + i), 1);
         }
-        ptx::mbar_init(Q_FULL, C::NPROD);
-        ptx::mbar_init(Q_EMPTY, 1);
+        for (int i = 0; i < NV; ++i) {
+            ptx::mbar_init(BAR(C::B_VFULL + i), 128);
+            ptx::mbar_init(BAR(C::B_VEMPTY + i), 1);
+        }
+        ptx::mbar_init(BAR(C::B_QFULL), 1);
+        ptx::mbar_init(BAR(C::B_QEMPTY), 1);
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(S_FULL(i), 1);
-            ptx::mbar_init(S_FREE(i), 128);
-            ptx::mbar_init(P_FULL(i), 128);
-            ptx::mbar_init(O_DONE(i), 1);
+            ptx::mbar_init(BAR(C::B_SFULL + i), 1);
+            ptx::mbar_init(BAR(C::B_SFREE + i), 256);
+            ptx::mbar_init(BAR(C::B_ODONE + i), 1);
         }
-        ptx::mbar_init(DRAIN, 1);
+        for (int i = 0; i < NP; ++i) ptx::mbar_init(BAR(C::B_PFULL + i), 256);
+        ptx::mbar_init(BAR(C::B_DRAIN), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -213,146 +257,227 @@ __global__ void __launch_bounds__(256, 1) fgattn_fwd_kernel(const FwdParams p) {
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + C::OFF_TMEM);
-    const uint32_t tS0 = tmem;                 // S^T slots: columns [0, MQ) and [MQ, 2MQ)
-    const uint32_t tO = tmem + 2u * MQ;        // O^T accumulator: columns [2MQ, 3MQ)
-
+    const uint32_t tS0 = tmem;           // S^T slots: columns [0, MQ) and [MQ, 2MQ)
+    const uint32_t tO = tmem + 2u * MQ;  // O^T accumulator: columns [2MQ, 3MQ)
     const int64_t L = p.L;
 
-    if (warp >= 4 && warp < 7) {
-        // ===================================================== producer (gathers)
-        const int u = threadIdx.x - 128;
-        int32_t* idx_smem = reinterpret_cast<int32_t*>(smem + C::OFF_IDX);
-        int64_t g = 0;
-        int64_t it = 0;
-        for (int64_t item = blockIdx.x; item < p.items; item += gridDim.x, ++it) {
+    if (warp >= 8 && warp < 11) {
+        // ===================================================== K producer (TMA)
+        if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
+        const int kw = warp - 8;
+        const int g4 = kw * 11 + lane;            // the chunk's 32 four-row groups: 11 + 11 + 10
+        const bool issuer = lane < 11 && g4 < 32;
+        const int my_groups = kw < 2 ? 11 : 10;
+        int64_t g = 0, it = 0;
+        int64_t issued = 0;    // chunks whose loads this warp has issued
+        int64_t q_issued = 0;  // query tiles issued (warp 8)
+        bool ok = true;
+        for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
             const int64_t bh = item / p.QB;
             const int64_t qb = item - bh * p.QB;
-            const int64_t cnt = item_count(p, item, u == 0);
+            const int64_t cnt = item_count(p, item, warp == 8 && lane == 0);
             const int64_t nch = (cnt + 127) / 128;
-            bool okq = it == 0 || bounded_wait(Q_EMPTY, (uint32_t)((it - 1) & 1), abort_flag);
-            okq = ptx::named_red_and(2, C::NPROD, okq);  // uniform exit: named barriers follow
-            if (!okq) break;
-            {  // query tile: MQ rows, zero-filled past L
-                const __nv_bfloat16* qsrc = p.q + (size_t)bh * L * D;
-                for (int id = u; id < MQ * C::PPR; id += C::NPROD) {
-                    const int row = id / C::PPR, pc = id % C::PPR;
-                    const int64_t grow = qb * MQ + row;
-                    const bool in = grow < L;
-                    const __nv_bfloat16* src = qsrc + (size_t)(in ? grow : 0) * D + pc * 8;
-                    const uint32_t dst = QTILE + (uint32_t)(pc / 8) * (MQ * 128) + swz(row, pc % 8, 128);
-                    ptx::cp_async_16(dst, src, in ? 16u : 0u);
-                }
-                ptx::cp_async_arrive_noinc(Q_FULL);
-            }
             const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
-            const __nv_bfloat16* kb = p.k + (size_t)bh * L * D;
-            const __nv_bfloat16* vb = p.v + (size_t)bh * L * D;
-            bool ok = true;
+            if (warp == 8) {  // the query tile (rows past L are padding; their results are never stored)
+                const bool okq = it == 0 || bounded_wait(BAR(C::B_QEMPTY), (uint32_t)((it - 1) & 1), abort_flag);
+                if (!__all_sync(0xffffffffu, okq)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(BAR(C::B_QFULL), (uint32_t)C::Q_TILE);
+#pragma unroll
+                    for (int pn = 0; pn < D / 64; ++pn)
+                        ptx::tma_load_2d(QTILE + (uint32_t)pn * (MQ * 128), &p.tmap_q, pn * 64,
+                                         (int32_t)(bh * L + qb * MQ), BAR(C::B_QFULL));
+                }
+                ++q_issued;
+                __syncwarp();
+            }
+            constexpr int PF = 4;  // index prefetch distance in chunks (the lists live in HBM)
+            int4 ring[PF];
+#pragma unroll
+            for (int i = 0; i < PF; ++i)
+                ring[i] = (issuer && i < nch) ? fetch_idx(lst, cnt, i, g4) : make_int4(0, 0, 0, 0);
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
-                const int st = (int)(gc % NST);
-                if (gc >= NST && !bounded_wait(KV_EMPTY(st), (uint32_t)((gc / NST - 1) & 1), abort_flag)) {
+                const int st = (int)(gc % NK);
+                const int4 cur = ring[0];
+#pragma unroll
+                for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
+                ring[PF - 1] = (issuer && c + PF < nch) ? fetch_idx(lst, cnt, c + PF, g4) : make_int4(0, 0, 0, 0);
+                const bool okw =
+                    gc < NK || bounded_wait(BAR(C::B_KEMPTY + st), (uint32_t)((gc / NK - 1) & 1), abort_flag);
+                if (!__all_sync(0xffffffffu, okw)) {
                     ok = false;
+                    break;
                 }
-                // the three producer warps agree before touching the stage
-                ok = ptx::named_red_and(2, C::NPROD, ok);
-                if (!ok) break;
-                int32_t* sidx = idx_smem + st * 128;
-                for (int r = u; r < 128; r += C::NPROD) {
-                    const int64_t j = c * 128 + r;
-                    int64_t idx = 0;  // rows past the list: any valid key (scores are masked)
-                    if (j < cnt) {
-                        idx = lst ? (int64_t)lst[j] : j;
-                        if (idx < 0 || idx >= L) {
-                            atomicOr(&g_device_error, kErrBadIndex);
-                            idx = 0;
-                        }
-                    }
-                    sidx[r] = (int32_t)idx;
+                if (lane == 0) ptx::mbar_arrive_expect_tx(BAR(C::B_KFULL + st), (uint32_t)(my_groups * 4 * D * 2));
+                __syncwarp();
+                if (issuer) {
+                    int32_t rows[4];
+                    rows_of(p, cur, bh * L, true, rows);
+                    const uint32_t dst = KSLOT(st) + (uint32_t)g4 * 512u;
+#pragma unroll
+                    for (int pn = 0; pn < D / 64; ++pn)
+                        ptx::tma_gather4(dst + (uint32_t)pn * (128 * 128), &p.tmap_k, pn * 64, rows[0], rows[1], rows[2],
+                                         rows[3], BAR(C::B_KFULL + st));
                 }
-                ptx::named_sync(2, C::NPROD);
-                const uint32_t kdst = KSLOT(st), vdst = VSLOT(st);
-#pragma unroll 2
-                for (int pid = u; pid < 128 * C::PPR; pid += C::NPROD) {
-                    const int r = pid / C::PPR, pc = pid % C::PPR;
-                    const size_t src = (size_t)sidx[r] * D + pc * 8;
-                    const uint32_t off = (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128);
-                    ptx::cp_async_16(kdst + off, kb + src, 16u);
-                    ptx::cp_async_16(vdst + off, vb + src, 16u);
-                }
-                ptx::cp_async_arrive_noinc(KV_FULL(st));
+                ++issued;
             }
-            if (!ok) break;
+            g += nch;
+        }
+        // Before the block exits, every load this warp issued has landed (on the normal
+        // path they all have already been consumed, so these waits return at once).
+        for (int64_t i = issued > NK ? issued - NK : 0; i < issued; ++i)
+            bounded_wait(BAR(C::B_KFULL + (int)(i % NK)), (uint32_t)((i / NK) & 1), abort_flag, false);
+        if (q_issued > 0) bounded_wait(BAR(C::B_QFULL), (uint32_t)((q_issued - 1) & 1), abort_flag, false);
+    } else if (warp >= 12) {
+        // ===================================================== V producer (cp.async)
+        if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
+        const int vw = warp - 12;  // rows [32*vw, 32*vw + 32) of each chunk
+        constexpr int PPR = D / 8;        // 16-byte pieces per row
+        constexpr int RPI = 32 / PPR;     // rows per warp instruction
+        int64_t g = 0;
+        bool ok = true;
+        for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
+            const int64_t bh = item / p.QB;
+            const int64_t cnt = item_count(p, item, false);
+            const int64_t nch = (cnt + 127) / 128;
+            const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
+            const __nv_bfloat16* vb = p.v_base + (size_t)bh * L * D;
+            auto fetch1 = [&](int64_t c) -> int32_t {
+                const int64_t j = c * 128 + vw * 32 + lane;
+                if (j >= cnt) return 0;
+                return lst ? __ldg(lst + j) : (int32_t)j;
+            };
+            constexpr int PF = 4;
+            int32_t ring[PF];
+#pragma unroll
+            for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch1(i) : 0;
+            for (int64_t c = 0; c < nch; ++c) {
+                const int64_t gc = g + c;
+                const int st = (int)(gc % NV);
+                int32_t idx = ring[0];
+#pragma unroll
+                for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
+                ring[PF - 1] = c + PF < nch ? fetch1(c + PF) : 0;
+                const bool okw =
+                    gc < NV || bounded_wait(BAR(C::B_VEMPTY + st), (uint32_t)((gc / NV - 1) & 1), abort_flag);
+                if (!__all_sync(0xffffffffu, okw)) {
+                    ok = false;
+                    break;
+                }
+                if (idx < 0 || (int64_t)idx >= L) {
+                    atomicOr(&g_device_error, kErrBadIndex);
+                    idx = 0;
+                }
+                const uint32_t vdst = VSLOT(st);
+#pragma unroll
+                for (int i = 0; i < 32 / RPI; ++i) {
+                    const int rl = i * RPI + lane / PPR;
+                    const int pc = lane % PPR;
+                    const int32_t ridx = __shfl_sync(0xffffffffu, idx, rl);
+                    const int r = vw * 32 + rl;
+                    ptx::cp_async_16(vdst + (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128),
+                                     vb + (size_t)ridx * D + pc * 8, 16u);
+                }
+                ptx::cp_async_arrive_noinc(BAR(C::B_VFULL + st));
+            }
             g += nch;
         }
         ptx::cp_async_wait_all();
-    } else if (warp == 7) {
+    } else if (warp == 11) {
         // ===================================================== MMA issuer
+        if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
         if (lane == 0) {
             constexpr uint32_t IDESC1 = umma_idesc_bf16(128, MQ, false, false);
             constexpr uint32_t IDESC2 = umma_idesc_bf16(D, MQ, true, true);
             constexpr uint32_t P_LAYOUT = (C::P_ROW == 128) ? 2u : (C::P_ROW == 64) ? 4u : 6u;
             bool ok = true;
             auto issue_pv = [&](int64_t gm, int64_t cm) -> bool {
-                const int st = (int)(gm % NST);
-                const int s = (int)(gm & 1);
-                if (!bounded_wait(P_FULL(s), (uint32_t)((gm >> 1) & 1), abort_flag)) return false;
+                const int vs = (int)(gm % NV);
+                const int pb = (int)(gm % NP);
+                if (!bounded_wait(BAR(C::B_VFULL + vs), (uint32_t)((gm / NV) & 1), abort_flag)) return false;
+                if (!bounded_wait(BAR(C::B_PFULL + pb), (uint32_t)((gm / NP) & 1), abort_flag)) return false;
                 ptx::tc_fence_after();
                 ptx::fence_proxy_async_smem();
-#pragma unroll
+#pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = umma_desc(VSLOT(st) + kk * 2048u, 128u * 128u, 1024u, 2u);
-                    const uint64_t bd = umma_desc(KSLOT(st) + kk * 16u * C::P_ROW, (uint32_t)C::P_PANEL,
-                                                  8u * C::P_ROW, P_LAYOUT);
+                    const uint64_t ad = umma_desc(VSLOT(vs) + kk * 2048u, 128u * 128u, 1024u, 2u);
+                    const uint64_t bd =
+                        umma_desc(PBUF(pb) + kk * 16u * C::P_ROW, (uint32_t)C::P_PANEL, 8u * C::P_ROW, P_LAYOUT);
                     ptx::mma_bf16_ss(tO, ad, bd, IDESC2, (cm > 0 || kk > 0) ? 1u : 0u);
                 }
-                ptx::mma_commit(KV_EMPTY(st));
-                ptx::mma_commit(O_DONE(s));
+                ptx::mma_commit(BAR(C::B_VEMPTY + vs));
+                ptx::mma_commit(BAR(C::B_ODONE + (int)(gm & 1)));
                 return true;
             };
-            int64_t g = 0;
-            int64_t it = 0;
+            int64_t g = 0, it = 0;
             for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
                 const int64_t nch = (item_count(p, item, false) + 127) / 128;
                 for (int64_t c = 0; c < nch; ++c) {
                     const int64_t gc = g + c;
-                    const int st = (int)(gc % NST);
+                    const int ks = (int)(gc % NK);
                     const int s = (int)(gc & 1);
-                    if (c == 0 && !bounded_wait(Q_FULL, (uint32_t)(it & 1), abort_flag)) { ok = false; break; }
-                    if (!bounded_wait(KV_FULL(st), (uint32_t)((gc / NST) & 1), abort_flag)) { ok = false; break; }
-                    if (gc >= 2 && !bounded_wait(S_FREE(s), (uint32_t)(((gc >> 1) - 1) & 1), abort_flag)) {
+                    if (c == 0 && !bounded_wait(BAR(C::B_QFULL), (uint32_t)(it & 1), abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!bounded_wait(BAR(C::B_KFULL + ks), (uint32_t)((gc / NK) & 1), abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (gc >= 2 &&
+                        !bounded_wait(BAR(C::B_SFREE + s), (uint32_t)(((gc >> 1) - 1) & 1), abort_flag)) {
                         ok = false;
                         break;
                     }
                     ptx::tc_fence_after();
-                    ptx::fence_proxy_async_smem();
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t koff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
                         const uint32_t qoff = (uint32_t)(kk / 4) * (MQ * 128) + (uint32_t)(kk % 4) * 32u;
-                        const uint64_t ad = umma_desc(KSLOT(st) + koff, 16u, 1024u, 2u);
+                        const uint64_t ad = umma_desc(KSLOT(ks) + koff, 16u, 1024u, 2u);
                         const uint64_t bd = umma_desc(QTILE + qoff, 16u, 1024u, 2u);
                         ptx::mma_bf16_ss(tS0 + (uint32_t)s * MQ, ad, bd, IDESC1, kk > 0 ? 1u : 0u);
                     }
-                    ptx::mma_commit(S_FULL(s));
-                    if (c == nch - 1) ptx::mma_commit(Q_EMPTY);
-                    if (c >= 1 && !issue_pv(gc - 1, c - 1)) { ok = false; break; }
+                    ptx::mma_commit(BAR(C::B_KEMPTY + ks));
+                    ptx::mma_commit(BAR(C::B_SFULL + s));
+                    if (c == nch - 1) ptx::mma_commit(BAR(C::B_QEMPTY));
+                    if (c >= 1 && !issue_pv(gc - 1, c - 1)) {
+                        ok = false;
+                        break;
+                    }
                 }
                 if (!ok) break;
-                if (!issue_pv(g + nch - 1, nch - 1)) { ok = false; break; }
+                if (!issue_pv(g + nch - 1, nch - 1)) {
+                    ok = false;
+                    break;
+                }
                 g += nch;
             }
             // drain: every MMA this thread issued has completed before TMEM is freed
-            ptx::mma_commit(DRAIN);
-            bounded_wait(DRAIN, 0u, abort_flag, /*honour_abort=*/false);
+            ptx::mma_commit(BAR(C::B_DRAIN));
+            bounded_wait(BAR(C::B_DRAIN), 0u, abort_flag, /*honour_abort=*/false);
         }
         __syncwarp();
     } else {
-        // ===================================================== softmax / epilogue
-        const int t = threadIdx.x;  // key lane within a chunk; TMEM lane t
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // ===================================================== softmax / epilogue (two warpgroups)
+        if constexpr (C::SOFT_REGS != 128) ptx::regs_inc<C::SOFT_REGS>();
+        const int wg = warp >> 2;         // 0 or 1
+        const int wq = warp & 3;          // warp within the group = TMEM lane quarter
+        const int t = threadIdx.x & 127;  // key lane within a chunk; TMEM lane t
+        const uint32_t nbar = 1u + (uint32_t)wg;
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        const uint32_t col0 = (uint32_t)(wg * CW);  // this group's first query column
         // d index held by this thread in the O^T accumulator (M = D layout)
-        const int dt = (D == 128) ? t : ((lane < 16) ? warp * 16 + lane : -1);
+        const int dt = (D == 128) ? t : ((lane < 16) ? wq * 16 + lane : -1);
+        float* mref = reinterpret_cast<float*>(smem + C::OFF_MREF) + wg * CW;
+        float* alpha = reinterpret_cast<float*>(smem + C::OFF_ALPHA) + wg * CW;
+        float* lfin = reinterpret_cast<float*>(smem + C::OFF_LFIN) + wg * CW;
+        float* red = reinterpret_cast<float*>(smem + C::OFF_RED) + wg * 4 * CW;
+        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem + C::OFF_STAGE + wg * C::STAGE);
         const float cs = p.scale_log2;
         int64_t g = 0;
         for (int64_t item = blockIdx.x; item < p.items; item += gridDim.x) {
@@ -360,182 +485,185 @@ __global__ void __launch_bounds__(256, 1) fgattn_fwd_kernel(const FwdParams p) {
             const int64_t qb = item - bh * p.QB;
             const int64_t cnt = item_count(p, item, false);
             const int64_t nch = (cnt + 127) / 128;
-            if (t < MQ) mref[t] = -INFINITY;
-            float lp[MQ];
+            if (t < CW) mref[t] = -INFINITY;
+            float lp[CW];
 #pragma unroll
-            for (int q = 0; q < MQ; ++q) lp[q] = 0.f;
-            ptx::named_sync(1, 128);
+            for (int q = 0; q < CW; ++q) lp[q] = 0.f;
+            ptx::named_sync(nbar, 128);
             bool ok = true;
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
                 const int s = (int)(gc & 1);
-                const int st = (int)(gc % NST);
-                ok = bounded_wait(S_FULL(s), (uint32_t)((gc >> 1) & 1), abort_flag);
-                ok = ptx::named_red_and(1, 128, ok);
+                const int pb = (int)(gc % NP);
+                ok = bounded_wait(BAR(C::B_SFULL + s), (uint32_t)((gc >> 1) & 1), abort_flag);
+                ok = ptx::named_red_and(nbar, 128, ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                float v[CW];
+                {
+                    const uint32_t ta = tS0 + (uint32_t)s * MQ + col0 + lane_base;
+                    if constexpr (CW >= 32) {
+#pragma unroll
+                        for (int pi = 0; pi < CW / 32; ++pi) {
+                            float tmp[32];
+                            ptx::tmem_ld32(ta + pi * 32, tmp);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[pi * 32 + j] = tmp[j];
+                        }
+                    } else if constexpr (CW == 16) {
+                        float tmp[16];
+                        ptx::tmem_ld16(ta, tmp);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) v[j] = tmp[j];
+                    } else {
+                        float tmp[8];
+                        ptx::tmem_ld8(ta, tmp);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) v[j] = tmp[j];
+                    }
+                    ptx::tmem_wait_ld();
+                }
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(BAR(C::B_SFREE + s));
                 const bool valid = c * 128 + t < cnt;
-                const uint32_t tS = tS0 + (uint32_t)s * MQ + lane_base;
-                float xs[C::KEEP ? MQ : 1];
-                // ---- pass 1: scores (log2 units) and the largest excess over the reference
+                // ---- largest excess of this key's scores over the references (log2 units)
                 float dmax = -INFINITY;
 #pragma unroll
-                for (int pi = 0; pi < MQ / 16; ++pi) {
-                    float v[16];
-                    ptx::tmem_ld16(tS + pi * 16, v);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float x = valid ? v[j] * cs : -INFINITY;
-                        if constexpr (C::KEEP) xs[pi * 16 + j] = x;
-                        dmax = fmaxf(dmax, x - mref[pi * 16 + j]);
-                    }
+                for (int q = 0; q < CW; q += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4*>(mref + q);
+                    dmax = ptx::max3(dmax, fmaf(v[q], cs, -m4.x), fmaf(v[q + 1], cs, -m4.y));
+                    dmax = ptx::max3(dmax, fmaf(v[q + 2], cs, -m4.z), fmaf(v[q + 3], cs, -m4.w));
                 }
-                if constexpr (C::KEEP) {
-                    ptx::tc_fence_before();
-                    ptx::mbar_arrive(S_FREE(s));
-                }
-                const bool need = ptx::named_red_or(1, 128, valid && dmax > TAU);
+                const bool need = ptx::named_red_or(nbar, 128, valid && dmax > TAU);
                 if (need) {
-                    // ---- exact column maxima of this chunk -> new references
+                    // ---- exact column maxima of this chunk -> raised references
 #pragma unroll
-                    for (int pi = 0; pi < MQ / 16; ++pi) {
-                        float v[16];
-                        if constexpr (!C::KEEP) {
-                            ptx::tmem_ld16(tS + pi * 16, v);
-                            ptx::tmem_wait_ld();
-                        }
+                    for (int q = 0; q < CW; ++q) {
+                        float x = valid ? v[q] * cs : -INFINITY;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            float x;
-                            if constexpr (C::KEEP) x = xs[pi * 16 + j];
-                            else x = valid ? v[j] * cs : -INFINITY;
-#pragma unroll
-                            for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-                            if (lane == ((pi * 16 + j) & 31)) red[warp * MQ + pi * 16 + j] = x;
-                        }
+                        for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+                        if (lane == (q & 31)) red[wq * CW + q] = x;
                     }
-                    ptx::named_sync(1, 128);
-                    if (t < MQ) {
+                    ptx::named_sync(nbar, 128);
+                    if (t < CW) {
                         const float mo = mref[t];
-                        const float mn = fmaxf(mo, fmaxf(fmaxf(red[t], red[MQ + t]), fmaxf(red[2 * MQ + t], red[3 * MQ + t])));
+                        const float mn =
+                            fmaxf(mo, fmaxf(fmaxf(red[t], red[CW + t]), fmaxf(red[2 * CW + t], red[3 * CW + t])));
                         alpha[t] = ptx::ex2(mo - mn);
                         mref[t] = mn;
                     }
-                    ptx::named_sync(1, 128);
+                    ptx::named_sync(nbar, 128);
 #pragma unroll
-                    for (int q = 0; q < MQ; ++q) lp[q] *= alpha[q];
+                    for (int q = 0; q < CW; ++q) lp[q] *= alpha[q];
                     if (c > 0) {
-                        // O holds chunks < c: wait for the last of them, then rescale its columns
+                        // O holds this item's chunks < c: wait for the last of them, rescale our columns
                         const int64_t gp = gc - 1;
-                        ok = bounded_wait(O_DONE((int)(gp & 1)), (uint32_t)((gp >> 1) & 1), abort_flag);
-                        ok = ptx::named_red_and(1, 128, ok);
+                        ok = bounded_wait(BAR(C::B_ODONE + (int)(gp & 1)), (uint32_t)((gp >> 1) & 1), abort_flag);
+                        ok = ptx::named_red_and(nbar, 128, ok);
                         if (!ok) break;
                         ptx::tc_fence_after();
 #pragma unroll
-                        for (int pi = 0; pi < MQ / 16; ++pi) {
-                            float o[16];
-                            ptx::tmem_ld16(tO + lane_base + pi * 16, o);
+                        for (int q0 = 0; q0 < CW; q0 += 8) {
+                            float o[8];
+                            ptx::tmem_ld8(tO + col0 + q0 + lane_base, o);
                             ptx::tmem_wait_ld();
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) o[j] *= alpha[pi * 16 + j];
-                            ptx::tmem_st16(tO + lane_base + pi * 16, o);
+                            for (int j = 0; j < 8; ++j) o[j] *= alpha[q0 + j];
+                            ptx::tmem_st8(tO + col0 + q0 + lane_base, o);
                         }
                         ptx::tmem_wait_st();
                     }
                 }
-                // ---- pass 2: probabilities -> bf16 P^T rows (this thread's key) in the K slot
-                const uint32_t prow = KSLOT(st);
+                if (!valid) {
 #pragma unroll
-                for (int pi = 0; pi < MQ / 16; ++pi) {
-                    float v[16];
-                    if constexpr (!C::KEEP) {
-                        ptx::tmem_ld16(tS + pi * 16, v);
-                        ptx::tmem_wait_ld();
-                    }
-                    uint32_t packed[8];
+                    for (int q = 0; q < CW; ++q) v[q] = -INFINITY;
+                }
+                // ---- the P buffer is free once the MMA that last read it has completed
+                if (gc >= NP) {
+                    const int64_t gr = gc - NP;
+                    ok = bounded_wait(BAR(C::B_ODONE + (int)(gr & 1)), (uint32_t)((gr >> 1) & 1), abort_flag);
+                    ok = ptx::named_red_and(nbar, 128, ok);
+                    if (!ok) break;
+                }
+                // ---- probabilities -> bf16 P^T row of this key, our query columns
+                const uint32_t prow = PBUF(pb);
 #pragma unroll
-                    for (int j = 0; j < 16; j += 2) {
-                        float x0, x1;
-                        if constexpr (C::KEEP) {
-                            x0 = xs[pi * 16 + j];
-                            x1 = xs[pi * 16 + j + 1];
-                        } else {
-                            x0 = valid ? v[j] * cs : -INFINITY;
-                            x1 = valid ? v[j + 1] * cs : -INFINITY;
-                        }
-                        const float p0 = ptx::ex2(x0 - mref[pi * 16 + j]);
-                        const float p1 = ptx::ex2(x1 - mref[pi * 16 + j + 1]);
-                        lp[pi * 16 + j] += p0;
-                        lp[pi * 16 + j + 1] += p1;
+                for (int q = 0; q < CW; q += 8) {
+                    const float4 ma = *reinterpret_cast<const float4*>(mref + q);
+                    const float4 mb = *reinterpret_cast<const float4*>(mref + q + 4);
+                    const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+                    uint32_t packed[4];
+#pragma unroll
+                    for (int j = 0; j < 8; j += 2) {
+                        const float p0 = ptx::ex2(fmaf(v[q + j], cs, -mm[j]));
+                        const float p1 = ptx::ex2(fmaf(v[q + j + 1], cs, -mm[j + 1]));
+                        lp[q + j] += p0;
+                        lp[q + j + 1] += p1;
                         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                         packed[j / 2] = *reinterpret_cast<uint32_t*>(&h);
                     }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int chunk = pi * 2 + h;  // 16-byte chunk = 8 queries
-                        const int panel = chunk / C::P_CPR;
-                        const uint32_t addr = prow + (uint32_t)panel * C::P_PANEL + swz(t, chunk % C::P_CPR, C::P_ROW);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[4 * h]),
-                                     "r"(packed[4 * h + 1]), "r"(packed[4 * h + 2]), "r"(packed[4 * h + 3])
-                                     : "memory");
-                    }
-                }
-                if constexpr (!C::KEEP) {
-                    ptx::tc_fence_before();
-                    ptx::mbar_arrive(S_FREE(s));
+                    const int chunk = (int)(col0 + q) / 8;  // 16-byte chunk = 8 queries
+                    const int panel = chunk / C::P_CPR;
+                    const uint32_t addr = prow + (uint32_t)panel * C::P_PANEL + swz(t, chunk % C::P_CPR, C::P_ROW);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[0]),
+                                 "r"(packed[1]), "r"(packed[2]), "r"(packed[3])
+                                 : "memory");
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(P_FULL(s));
+                ptx::mbar_arrive(BAR(C::B_PFULL + pb));
             }
             if (!ok) break;
-            // ===================== epilogue: O / l -> bf16 rows, lse
+            // ===================== epilogue: O / l -> bf16 rows, lse (our query columns)
             const int64_t e = g + nch - 1;
-            ok = bounded_wait(O_DONE((int)(e & 1)), (uint32_t)((e >> 1) & 1), abort_flag);
-            ok = ptx::named_red_and(1, 128, ok);
+            ok = bounded_wait(BAR(C::B_ODONE + (int)(e & 1)), (uint32_t)((e >> 1) & 1), abort_flag);
+            ok = ptx::named_red_and(nbar, 128, ok);
             if (!ok) break;
             ptx::tc_fence_after();
 #pragma unroll
-            for (int q = 0; q < MQ; ++q) {
+            for (int q = 0; q < CW; ++q) {
                 float x = lp[q];
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                if (lane == (q & 31)) red[warp * MQ + q] = x;
+                if (lane == (q & 31)) red[wq * CW + q] = x;
             }
-            ptx::named_sync(1, 128);
-            if (t < MQ) {
-                const float l = (red[t] + red[MQ + t]) + (red[2 * MQ + t] + red[3 * MQ + t]);
+            ptx::named_sync(nbar, 128);
+            if (t < CW) {
+                const float l = (red[t] + red[CW + t]) + (red[2 * CW + t] + red[3 * CW + t]);
                 lfin[t] = 1.0f / l;
-                const int64_t row = qb * MQ + t;
+                const int64_t row = qb * MQ + col0 + t;
                 if (p.lse != nullptr && row < L) {
                     float lg;
                     asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l));
                     p.lse[bh * L + row] = (mref[t] + lg) * 0.69314718055994530942f;
                 }
             }
-            ptx::named_sync(1, 128);
-            __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem + C::OFF_STAGE);
+            ptx::named_sync(nbar, 128);
             __nv_bfloat16* outb = p.out + (size_t)bh * L * D;
+            constexpr int SR = C::SROWS;
 #pragma unroll 1
-            for (int pi = 0; pi < MQ / 16; ++pi) {
-                float o[16];
-                ptx::tmem_ld16(tO + lane_base + pi * 16, o);
+            for (int q0 = 0; q0 < CW; q0 += SR) {
+                float o[SR];
+                if constexpr (SR == 16) {
+                    ptx::tmem_ld16(tO + col0 + q0 + lane_base, o);
+                } else {
+                    ptx::tmem_ld8(tO + col0 + q0 + lane_base, o);
+                }
                 ptx::tmem_wait_ld();
                 if (dt >= 0) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) stage[j * D + dt] = __float2bfloat16_rn(o[j] * lfin[pi * 16 + j]);
+                    for (int j = 0; j < SR; ++j) stage[j * D + dt] = __float2bfloat16_rn(o[j] * lfin[q0 + j]);
                 }
-                ptx::named_sync(1, 128);
-                for (int vi = t; vi < 16 * C::PPR; vi += 128) {
-                    const int r = vi / C::PPR, pc = vi % C::PPR;
-                    const int64_t row = qb * MQ + pi * 16 + r;
+                ptx::named_sync(nbar, 128);
+                for (int vi = t; vi < SR * (D / 8); vi += 128) {
+                    const int r = vi / (D / 8), pc = vi % (D / 8);
+                    const int64_t row = qb * MQ + col0 + q0 + r;
                     if (row < L) {
                         const uint4 val = *reinterpret_cast<const uint4*>(stage + r * D + pc * 8);
                         *reinterpret_cast<uint4*>(outb + row * D + pc * 8) = val;
                     }
                 }
-                ptx::named_sync(1, 128);
+                ptx::named_sync(nbar, 128);
             }
             ptx::tc_fence_before();
             g += nch;
@@ -545,7 +673,7 @@ __global__ void __launch_bounds__(256, 1) fgattn_fwd_kernel(const FwdParams p) {
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (warp == 7) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == 11) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace fgattn

@@ -14,6 +14,37 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// cuTensorMapEncodeTiled, fetched through the runtime so the library needs no -lcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// Row-major bf16 matrix [rows][d] viewed in boxes of 64 columns x box_rows rows, 128B swizzle.
+bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t d, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {64u, box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int current_sms() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -23,8 +54,12 @@ int current_sms() {
 }
 
 template <int D, int MQ>
-fgattn_status launch_fwd(const fgattn::FwdParams& prm, cudaStream_t stream) {
+fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const void* k, const void* v, int64_t rows,
+                         cudaStream_t stream) {
     using C = fgattn::FwdCfg<D, MQ>;
+    if (!encode_rows(&prm.tmap_q, q, rows, D, MQ) || !encode_rows(&prm.tmap_k, k, rows, D, 1))
+        return FGATTN_ERR_CUDA;
+    prm.v_base = static_cast<const __nv_bfloat16*>(v);
     // Request enough shared memory that exactly one block is resident per SM:
     // the grid is persistent (one block per SM, static round-robin over work).
     const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;
@@ -78,16 +113,14 @@ fgattn_status fgattn_forward(const void* q, const void* k, const void* v, const 
     if (L > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return FGATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FGATTN_ERR_INVALID_ARG;
-    if (kept_idx && (reinterpret_cast<uintptr_t>(kept_idx) & 3u)) return FGATTN_ERR_INVALID_ARG;
+    if (kept_idx && !aligned16(kept_idx)) return FGATTN_ERR_INVALID_ARG;  // rows are read as int4
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FGATTN_ERR_INVALID_ARG;
-    if (kept_idx && cap < L) return FGATTN_ERR_CAPACITY;
+    if (kept_idx && (cap < L || (cap & 3))) return FGATTN_ERR_CAPACITY;
     if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
     if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
 
+    if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
     fgattn::FwdParams prm;
-    prm.q = static_cast<const __nv_bfloat16*>(q);
-    prm.k = static_cast<const __nv_bfloat16*>(k);
-    prm.v = static_cast<const __nv_bfloat16*>(v);
     prm.kept_idx = kept_idx;
     prm.kept_cnt = kept_cnt;
     prm.out = static_cast<__nv_bfloat16*>(out);
@@ -100,19 +133,20 @@ fgattn_status fgattn_forward(const void* q, const void* k, const void* v, const 
     (void)N;  // the key lists already encode the tile width
 
     cudaStream_t s = (cudaStream_t)stream;
+    const int64_t rows = B * H * L;
     if (d == 128) {
         switch (M) {
-            case 16: return launch_fwd<128, 16>(prm, s);
-            case 32: return launch_fwd<128, 32>(prm, s);
-            case 64: return launch_fwd<128, 64>(prm, s);
-            default: return launch_fwd<128, 128>(prm, s);
+            case 16: return launch_fwd<128, 16>(prm, q, k, v, rows, s);
+            case 32: return launch_fwd<128, 32>(prm, q, k, v, rows, s);
+            case 64: return launch_fwd<128, 64>(prm, q, k, v, rows, s);
+            default: return launch_fwd<128, 128>(prm, q, k, v, rows, s);
         }
     }
     switch (M) {
-        case 16: return launch_fwd<64, 16>(prm, s);
-        case 32: return launch_fwd<64, 32>(prm, s);
-        case 64: return launch_fwd<64, 64>(prm, s);
-        default: return launch_fwd<64, 128>(prm, s);
+        case 16: return launch_fwd<64, 16>(prm, q, k, v, rows, s);
+        case 32: return launch_fwd<64, 32>(prm, q, k, v, rows, s);
+        case 64: return launch_fwd<64, 64>(prm, q, k, v, rows, s);
+        default: return launch_fwd<64, 128>(prm, q, k, v, rows, s);
     }
 }
 

@@ -89,7 +89,8 @@ fgattn_status fgattn_compact_mask(const uint32_t* mask, int64_t B, int64_t H, in
  *   s_ij = scale * q_i . k_j,  p_ij = exp(s_ij - m_i),  l_i = sum_j p_ij,
  *   out_i = sum_j p_ij v_j / l_i  (stored as bf16),  lse_i = m_i + ln l_i.
  *   q, k, v   in   device bf16 [B][H][L][d]
- *   kept_idx  in   device int32 [B][H][QB][cap] (as written by fgattn_compact_mask,
+ *   kept_idx  in   device int32 [B][H][QB][cap], cap >= L, cap % 4 == 0
+ *                  (as written by fgattn_compact_mask,
  *                  or any ascending or unordered list of distinct keys < L),
  *                  or NULL for a dense run of the same kernel (every key kept)
  *   kept_cnt  in   device int32 [B][H][QB] (ignored when kept_idx is NULL);

@@ -81,6 +81,8 @@ def _cmp(**kw):
     (dict(q=P + 8), F.ERR_INVALID_ARG),
     (dict(lse=P + 2), F.ERR_INVALID_ARG),
     (dict(cap=63), F.ERR_CAPACITY),
+    (dict(cap=66), F.ERR_CAPACITY),
+    (dict(idx=P + 4), F.ERR_INVALID_ARG),
     (dict(d=96), F.ERR_UNSUPPORTED),
     (dict(d=256), F.ERR_UNSUPPORTED),
     (dict(M=48), F.ERR_UNSUPPORTED),
