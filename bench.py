@@ -71,11 +71,19 @@ def head_shard(H: int, rank: int) -> range:
 
 
 def reduce_max(x: float, dist) -> float:
+    """Max of a per-rank scalar (device time of the slowest rank)."""
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, flops_per_rank: float, max_ms_per_step: float) -> float:
+    """Whole-job effective TFLOP/s: every rank does the same work (weak scaling),
+    timed by the slowest rank."""
+    return world * flops_per_rank / (max_ms_per_step * 1e-3) / 1e12
 
 
 def barrier(dist):
@@ -311,7 +319,7 @@ def main():
     clocks = sampler.summary()
     assert F.device_error() == 0, "device error in the timed region"
     ms_per_step = total_ms / args.steps
-    value = world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(world, flops_per_step, ms_per_step)
 
     # ---- end to end through the public API: pinned host inputs -> device -> host results
     qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
@@ -341,13 +349,13 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1), dist) / args.e2e_steps
-    e2e_value = world * flops_per_step / (e2e_ms * 1e-3) / 1e12
+    e2e_value = job_throughput(world, flops_per_step, e2e_ms)
 
     # ---- roofline for the dominant kernel (the forward): tensor-bound on kept FLOPs
     peaks, peak_kind = load_peaks()
     achieved = flops_per_step / (fwd_ms * 1e-3) / 1e12
     from fine_grained_sparse_fgattn_b200 import _build
-    traffic, _ = ncu_traffic(w.name, _build.source_hash())
+    traffic, _ = ncu_traffic(w.name, _build.kernel_hash("fwd"))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                 "peak_kind": f"{peak_kind} bf16 burst", "kernel": "fgattn_fwd_kernel<128,64>",

@@ -29,6 +29,16 @@ def source_hash() -> str:
     return h.hexdigest()
 
 
+def kernel_hash(kernel: str) -> str:
+    """Hash of the sources one kernel is built from (ties a profile to a kernel version)."""
+    files = {"fwd": ["attention_fwd.cuh", "sm100_ptx.cuh"], "compact": ["compact_mask.cuh"]}[kernel]
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def is_current() -> bool:
     if not os.path.exists(LIB) or not os.path.exists(STAMP):
         return False

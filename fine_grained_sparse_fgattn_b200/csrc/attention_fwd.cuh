@@ -25,9 +25,13 @@
 // Warp roles (512 threads = four warpgroups):
 //   warps 0-3   softmax warpgroup 0: query columns [0, MQ/2)
 //   warps 4-7   softmax warpgroup 1: query columns [MQ/2, MQ)
-//   warps 8-10  K producer: TMA tile load of the query block, TMA gather4 of K rows
+//   warps 8-10  K producer: TMA tile load of the query block; K rows by TMA
 //   warp  11    TMEM allocation + single-thread tcgen05.mma issue
-//   warps 12-15 V producer: cp.async row gathers of V
+//   warps 12-15 V producer: V rows by TMA or cp.async
+// Each chunk is loaded as eight 16-row segments.  A segment whose 16 kept keys
+// are consecutive (always the case for key groups of N >= 16 keys, N a multiple
+// of 16) is one tiled TMA box; any other segment is gathered row by row (K with
+// TMA gather4, V with cp.async).
 // Gathering K and V through the two different copy paths (TMA and the LSU)
 // keeps more row requests in flight per SM than either path alone; the
 // producer warpgroups hand most of their registers to the softmax groups.
@@ -53,8 +57,10 @@ constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 
 struct alignas(64) FwdParams {
     CUtensorMap tmap_q;  // [B*H*L rows][D], box {64, MQ}, 128B swizzle
-    CUtensorMap tmap_k;  // [B*H*L rows][D], box {64, 1},  128B swizzle (row gathers)
-    const __nv_bfloat16* v_base;  // V rows, gathered with cp.async
+    CUtensorMap tmap_k;    // [B*H*L rows][D], box {64, 1},  128B swizzle (row gathers)
+    CUtensorMap tmap_k16;  // [B*H*L rows][D], box {64, 16}, 128B swizzle (16 consecutive rows)
+    CUtensorMap tmap_v16;  // same for V
+    const __nv_bfloat16* v_base;  // V rows, gathered with cp.async where not consecutive
     const int32_t* kept_idx;  // nullptr: dense (every key kept)
     const int32_t* kept_cnt;
     __nv_bfloat16* out;
@@ -265,9 +271,12 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
         // ===================================================== K producer (TMA)
         if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
         const int kw = warp - 8;
-        const int g4 = kw * 11 + lane;            // the chunk's 32 four-row groups: 11 + 11 + 10
-        const bool issuer = lane < 11 && g4 < 32;
-        const int my_groups = kw < 2 ? 11 : 10;
+        // segments 0-2 -> warp 8, 3-5 -> warp 9, 6-7 -> warp 10; four lanes (4-row groups) each
+        const int seg0 = kw * 3;
+        const int nseg = kw < 2 ? 3 : 2;
+        const int g4 = seg0 * 4 + lane;            // this lane's 4-row group in the chunk
+        const bool issuer = lane < nseg * 4;
+        const int lseg = lane >> 2;                // segment within the warp
         int64_t g = 0, it = 0;
         int64_t issued = 0;    // chunks whose loads this warp has issued
         int64_t q_issued = 0;  // query tiles issued (warp 8)
@@ -298,30 +307,47 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
             int4 ring[PF];
 #pragma unroll
             for (int i = 0; i < PF; ++i)
-                ring[i] = (issuer && i < nch) ? fetch_idx(lst, cnt, i, g4) : make_int4(0, 0, 0, 0);
+                ring[i] = (issuer && i < nch) ? fetch_idx(lst, cnt, i, g4) : make_int4(-1, -1, -1, -1);
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
                 const int st = (int)(gc % NK);
                 const int4 cur = ring[0];
 #pragma unroll
                 for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
-                ring[PF - 1] = (issuer && c + PF < nch) ? fetch_idx(lst, cnt, c + PF, g4) : make_int4(0, 0, 0, 0);
+                ring[PF - 1] = (issuer && c + PF < nch) ? fetch_idx(lst, cnt, c + PF, g4) : make_int4(-1, -1, -1, -1);
                 const bool okw =
                     gc < NK || bounded_wait(BAR(C::B_KEMPTY + st), (uint32_t)((gc / NK - 1) & 1), abort_flag);
                 if (!__all_sync(0xffffffffu, okw)) {
                     ok = false;
                     break;
                 }
-                if (lane == 0) ptx::mbar_arrive_expect_tx(BAR(C::B_KFULL + st), (uint32_t)(my_groups * 4 * D * 2));
+                // a segment is one TMA box when its 16 keys are real and consecutive
+                const int64_t j0 = c * 128 + 4 * g4;
+                const int32_t first = __shfl_sync(0xffffffffu, cur.x, lane & ~3);
+                const bool run = issuer && j0 + 3 < cnt && cur.x == first + 4 * (lane & 3) && cur.y == cur.x + 1 &&
+                                 cur.z == cur.x + 2 && cur.w == cur.x + 3 && first >= 0 && first + 15 < L;
+                const uint32_t runs = __ballot_sync(0xffffffffu, run);
+                const bool seg_run = ((runs >> (lseg * 4)) & 0xFu) == 0xFu;
+                if (lane == 0)
+                    ptx::mbar_arrive_expect_tx(BAR(C::B_KFULL + st), (uint32_t)(nseg * 16 * D * 2));
                 __syncwarp();
                 if (issuer) {
-                    int32_t rows[4];
-                    rows_of(p, cur, bh * L, true, rows);
                     const uint32_t dst = KSLOT(st) + (uint32_t)g4 * 512u;
+                    if (seg_run) {
+                        if ((lane & 3) == 0) {
 #pragma unroll
-                    for (int pn = 0; pn < D / 64; ++pn)
-                        ptx::tma_gather4(dst + (uint32_t)pn * (128 * 128), &p.tmap_k, pn * 64, rows[0], rows[1], rows[2],
-                                         rows[3], BAR(C::B_KFULL + st));
+                            for (int pn = 0; pn < D / 64; ++pn)
+                                ptx::tma_load_2d(dst + (uint32_t)pn * (128 * 128), &p.tmap_k16, pn * 64,
+                                                 (int32_t)(bh * L + first), BAR(C::B_KFULL + st));
+                        }
+                    } else {
+                        int32_t rows[4];
+                        rows_of(p, cur, bh * L, true, rows);
+#pragma unroll
+                        for (int pn = 0; pn < D / 64; ++pn)
+                            ptx::tma_gather4(dst + (uint32_t)pn * (128 * 128), &p.tmap_k, pn * 64, rows[0], rows[1],
+                                             rows[2], rows[3], BAR(C::B_KFULL + st));
+                    }
                 }
                 ++issued;
             }
@@ -333,11 +359,11 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
             bounded_wait(BAR(C::B_KFULL + (int)(i % NK)), (uint32_t)((i / NK) & 1), abort_flag, false);
         if (q_issued > 0) bounded_wait(BAR(C::B_QFULL), (uint32_t)((q_issued - 1) & 1), abort_flag, false);
     } else if (warp >= 12) {
-        // ===================================================== V producer (cp.async)
+        // ===================================================== V producer (TMA boxes / cp.async)
         if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
-        const int vw = warp - 12;  // rows [32*vw, 32*vw + 32) of each chunk
-        constexpr int PPR = D / 8;        // 16-byte pieces per row
-        constexpr int RPI = 32 / PPR;     // rows per warp instruction
+        const int vw = warp - 12;      // rows [32*vw, 32*vw + 32) of each chunk = two segments
+        constexpr int PPR = D / 8;     // 16-byte pieces per row
+        constexpr int RPI = 32 / PPR;  // rows per warp instruction
         int64_t g = 0;
         bool ok = true;
         for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
@@ -348,39 +374,55 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
             const __nv_bfloat16* vb = p.v_base + (size_t)bh * L * D;
             auto fetch1 = [&](int64_t c) -> int32_t {
                 const int64_t j = c * 128 + vw * 32 + lane;
-                if (j >= cnt) return 0;
+                if (j >= cnt) return -1;  // past the list
                 return lst ? __ldg(lst + j) : (int32_t)j;
             };
             constexpr int PF = 4;
             int32_t ring[PF];
 #pragma unroll
-            for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch1(i) : 0;
+            for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch1(i) : -1;
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
                 const int st = (int)(gc % NV);
                 int32_t idx = ring[0];
 #pragma unroll
                 for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
-                ring[PF - 1] = c + PF < nch ? fetch1(c + PF) : 0;
+                ring[PF - 1] = c + PF < nch ? fetch1(c + PF) : -1;
                 const bool okw =
                     gc < NV || bounded_wait(BAR(C::B_VEMPTY + st), (uint32_t)((gc / NV - 1) & 1), abort_flag);
                 if (!__all_sync(0xffffffffu, okw)) {
                     ok = false;
                     break;
                 }
-                if (idx < 0 || (int64_t)idx >= L) {
-                    atomicOr(&g_device_error, kErrBadIndex);
-                    idx = 0;
-                }
+                const int32_t first = __shfl_sync(0xffffffffu, idx, lane & 16);
+                const bool run = idx >= 0 && idx == first + (lane & 15) && first + 15 < L;
+                const uint32_t runs = __ballot_sync(0xffffffffu, run);
+                if (idx >= L) atomicOr(&g_device_error, kErrBadIndex);
+                if (idx < 0 || idx >= L) idx = 0;  // past the list, or corrupt: key 0 (scores are masked)
                 const uint32_t vdst = VSLOT(st);
 #pragma unroll
-                for (int i = 0; i < 32 / RPI; ++i) {
-                    const int rl = i * RPI + lane / PPR;
-                    const int pc = lane % PPR;
-                    const int32_t ridx = __shfl_sync(0xffffffffu, idx, rl);
-                    const int r = vw * 32 + rl;
-                    ptx::cp_async_16(vdst + (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128),
-                                     vb + (size_t)ridx * D + pc * 8, 16u);
+                for (int sg = 0; sg < 2; ++sg) {
+                    const int r0 = vw * 32 + sg * 16;
+                    if (((runs >> (16 * sg)) & 0xFFFFu) == 0xFFFFu) {
+                        const int32_t fs = __shfl_sync(0xffffffffu, first, 16 * sg);
+                        if (lane == 0) {
+                            ptx::mbar_expect_tx(BAR(C::B_VFULL + st), (uint32_t)(16 * D * 2));
+#pragma unroll
+                            for (int pn = 0; pn < D / 64; ++pn)
+                                ptx::tma_load_2d(vdst + (uint32_t)pn * (128 * 128) + (uint32_t)r0 * 128u, &p.tmap_v16,
+                                                 pn * 64, (int32_t)(bh * L + fs), BAR(C::B_VFULL + st));
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16 / RPI; ++i) {
+                            const int rl = sg * 16 + i * RPI + lane / PPR;
+                            const int pc = lane % PPR;
+                            const int32_t ridx = __shfl_sync(0xffffffffu, idx, rl);
+                            const int r = vw * 32 + rl;
+                            ptx::cp_async_16(vdst + (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128),
+                                             vb + (size_t)ridx * D + pc * 8, 16u);
+                        }
+                    }
                 }
                 ptx::cp_async_arrive_noinc(BAR(C::B_VFULL + st));
             }

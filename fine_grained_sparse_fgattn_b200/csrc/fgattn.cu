@@ -57,7 +57,8 @@ template <int D, int MQ>
 fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const void* k, const void* v, int64_t rows,
                          cudaStream_t stream) {
     using C = fgattn::FwdCfg<D, MQ>;
-    if (!encode_rows(&prm.tmap_q, q, rows, D, MQ) || !encode_rows(&prm.tmap_k, k, rows, D, 1))
+    if (!encode_rows(&prm.tmap_q, q, rows, D, MQ) || !encode_rows(&prm.tmap_k, k, rows, D, 1) ||
+        !encode_rows(&prm.tmap_k16, k, rows, D, 16) || !encode_rows(&prm.tmap_v16, v, rows, D, 16))
         return FGATTN_ERR_CUDA;
     prm.v_base = static_cast<const __nv_bfloat16*>(v);
     // Request enough shared memory that exactly one block is resident per SM:
@@ -93,14 +94,19 @@ fgattn_status fgattn_compact_mask(const uint32_t* mask, int64_t B, int64_t H, in
     if (L > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
     if (!aligned16(kept_idx) || (reinterpret_cast<uintptr_t>(mask) & 3u)) return FGATTN_ERR_INVALID_ARG;
     if (cap < L || (cap & 3)) return FGATTN_ERR_CAPACITY;
+    if (N > L) N = L;  // one key group either way (G = 1): same tiles, same keys
     const int64_t QB = (L + M - 1) / M;
     const int64_t G = (L + N - 1) / N;
     const int64_t W = (G + 31) / 32;
     const int64_t rows = B * H * QB;
     const int64_t blocks = (rows + 7) / 8;
     if (blocks > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
-    fgattn::compact_mask_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(mask, rows, QB, L, M, N, G, W,
-                                                                                      kept_idx, kept_cnt, cap);
+    if (N % 4 == 0)
+        fgattn::compact_mask_kernel<4><<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
+            mask, rows, QB, L, M, N, G, W, kept_idx, kept_cnt, cap);
+    else
+        fgattn::compact_mask_kernel<1><<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
+            mask, rows, QB, L, M, N, G, W, kept_idx, kept_cnt, cap);
     return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
 }
 
