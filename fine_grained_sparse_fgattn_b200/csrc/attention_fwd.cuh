@@ -92,8 +92,10 @@ struct FwdCfg {
         return nk * KV_TILE + nv * KV_TILE + np * P_TILE + Q_TILE + 2 * STAGE + MISC;
     }
     // pipeline depths: K ring, V ring, P buffers (deepest that fits)
-    static constexpr int NK = fixed_bytes(3, 2, 1) <= LIMIT ? 3 : 2;
-    static constexpr int NV = fixed_bytes(NK, 3, 2) <= LIMIT ? 3 : 2;
+    // The V ring has two stages so that "V slot free" is exactly "MMA2 of the chunk
+    // two back done" (o_done, no extra tensor-core commit); spare room deepens the K ring.
+    static constexpr int NV = 2;
+    static constexpr int NK = fixed_bytes(4, NV, 2) <= LIMIT ? 4 : fixed_bytes(3, NV, 1) <= LIMIT ? 3 : 2;
     static constexpr int NP = fixed_bytes(NK, NV, 2) <= LIMIT ? 2 : 1;
     static_assert(fixed_bytes(NK, NV, NP) <= LIMIT, "shared memory");
     static constexpr int OFF_K = 0;
@@ -106,8 +108,11 @@ struct FwdCfg {
     static constexpr int OFF_LFIN = OFF_ALPHA + 2 * CW * 4;  // [2][CW]
     static constexpr int OFF_RED = OFF_LFIN + 2 * CW * 4;    // [2][4][CW]
     static constexpr int OFF_BAR = (OFF_RED + 2 * 4 * CW * 4 + 7) / 8 * 8;
-    // barriers: k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] q_full q_empty
+    // barriers: k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] (unused: o_done serves) q_full q_empty
     //           s_full[2] s_free[2] p_full[NP] o_done[2] drain
+    // Only s_full and o_done are tensor-core commits (each commit costs tensor-pipe
+    // time); k_empty and q_empty are arrived by a softmax thread once s_full shows
+    // that the MMA reading them has finished.
     static constexpr int B_KFULL = 0, B_KEMPTY = NK, B_VFULL = 2 * NK, B_VEMPTY = 2 * NK + NV;
     static constexpr int B_QFULL = 2 * NK + 2 * NV, B_QEMPTY = B_QFULL + 1, B_SFULL = B_QFULL + 2;
     static constexpr int B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_ODONE = B_PFULL + NP;
@@ -388,8 +393,9 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
 #pragma unroll
                 for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
                 ring[PF - 1] = c + PF < nch ? fetch1(c + PF) : -1;
+                // slot (gc % 2) is free once MMA2 of chunk gc-2 has completed
                 const bool okw =
-                    gc < NV || bounded_wait(BAR(C::B_VEMPTY + st), (uint32_t)((gc / NV - 1) & 1), abort_flag);
+                    gc < 2 || bounded_wait(BAR(C::B_ODONE + (int)(gc & 1)), (uint32_t)(((gc - 2) >> 1) & 1), abort_flag);
                 if (!__all_sync(0xffffffffu, okw)) {
                     ok = false;
                     break;
@@ -451,51 +457,41 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
                         umma_desc(PBUF(pb) + kk * 16u * C::P_ROW, (uint32_t)C::P_PANEL, 8u * C::P_ROW, P_LAYOUT);
                     ptx::mma_bf16_ss(tO, ad, bd, IDESC2, (cm > 0 || kk > 0) ? 1u : 0u);
                 }
-                ptx::mma_commit(BAR(C::B_VEMPTY + vs));
                 ptx::mma_commit(BAR(C::B_ODONE + (int)(gm & 1)));
                 return true;
             };
+            // S^T of chunk gc into its slot (MMA1), once its K rows have landed and the
+            // softmax has copied the slot's previous contents (chunk gc-2) to registers.
+            auto issue_s = [&](int64_t gc, int64_t c, int64_t it) -> bool {
+                const int ks = (int)(gc % NK);
+                const int s = (int)(gc & 1);
+                if (c == 0 && !bounded_wait(BAR(C::B_QFULL), (uint32_t)(it & 1), abort_flag)) return false;
+                if (!bounded_wait(BAR(C::B_KFULL + ks), (uint32_t)((gc / NK) & 1), abort_flag)) return false;
+                if (gc >= 2 && !bounded_wait(BAR(C::B_SFREE + s), (uint32_t)(((gc >> 1) - 1) & 1), abort_flag))
+                    return false;
+                ptx::tc_fence_after();
+#pragma unroll 1
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
+                    const uint32_t qoff = (uint32_t)(kk / 4) * (MQ * 128) + (uint32_t)(kk % 4) * 32u;
+                    const uint64_t ad = umma_desc(KSLOT(ks) + koff, 16u, 1024u, 2u);
+                    const uint64_t bd = umma_desc(QTILE + qoff, 16u, 1024u, 2u);
+                    ptx::mma_bf16_ss(tS0 + (uint32_t)s * MQ, ad, bd, IDESC1, kk > 0 ? 1u : 0u);
+                }
+                ptx::mma_commit(BAR(C::B_SFULL + s));
+                return true;
+            };
+            // Issue order within an item: S of chunks 0 and 1, then for every chunk c
+            // the S of chunk c+2 (as soon as its slot frees, early in softmax(c)) before
+            // the P.V of chunk c (which waits for the end of softmax(c)).  The tensor core
+            // thus computes the next scores while the softmax works on the current ones.
             int64_t g = 0, it = 0;
             for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
                 const int64_t nch = (item_count(p, item, false) + 127) / 128;
-                for (int64_t c = 0; c < nch; ++c) {
-                    const int64_t gc = g + c;
-                    const int ks = (int)(gc % NK);
-                    const int s = (int)(gc & 1);
-                    if (c == 0 && !bounded_wait(BAR(C::B_QFULL), (uint32_t)(it & 1), abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!bounded_wait(BAR(C::B_KFULL + ks), (uint32_t)((gc / NK) & 1), abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (gc >= 2 &&
-                        !bounded_wait(BAR(C::B_SFREE + s), (uint32_t)(((gc >> 1) - 1) & 1), abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-#pragma unroll 1
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t koff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
-                        const uint32_t qoff = (uint32_t)(kk / 4) * (MQ * 128) + (uint32_t)(kk % 4) * 32u;
-                        const uint64_t ad = umma_desc(KSLOT(ks) + koff, 16u, 1024u, 2u);
-                        const uint64_t bd = umma_desc(QTILE + qoff, 16u, 1024u, 2u);
-                        ptx::mma_bf16_ss(tS0 + (uint32_t)s * MQ, ad, bd, IDESC1, kk > 0 ? 1u : 0u);
-                    }
-                    ptx::mma_commit(BAR(C::B_KEMPTY + ks));
-                    ptx::mma_commit(BAR(C::B_SFULL + s));
-                    if (c == nch - 1) ptx::mma_commit(BAR(C::B_QEMPTY));
-                    if (c >= 1 && !issue_pv(gc - 1, c - 1)) {
-                        ok = false;
-                        break;
-                    }
-                }
-                if (!ok) break;
-                if (!issue_pv(g + nch - 1, nch - 1)) {
-                    ok = false;
-                    break;
+                for (int64_t c = 0; c < nch && c < 2 && ok; ++c) ok = issue_s(g + c, c, it);
+                for (int64_t c = 0; c < nch && ok; ++c) {
+                    if (c + 2 < nch) ok = issue_s(g + c + 2, c + 2, it);
+                    if (ok) ok = issue_pv(g + c, c);
                 }
                 g += nch;
             }
@@ -541,6 +537,12 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
                 ok = ptx::named_red_and(nbar, 128, ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                if (wg == 0 && t == 0) {
+                    // MMA1 of this chunk has finished reading its K slot (and, for the
+                    // item's last chunk, the query tile)
+                    ptx::mbar_arrive(BAR(C::B_KEMPTY + (int)(gc % NK)));
+                    if (c == nch - 1) ptx::mbar_arrive(BAR(C::B_QEMPTY));
+                }
                 float v[CW];
                 {
                     const uint32_t ta = tS0 + (uint32_t)s * MQ + col0 + lane_base;
