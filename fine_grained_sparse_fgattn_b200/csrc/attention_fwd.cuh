@@ -528,14 +528,15 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
 #pragma unroll
             for (int q = 0; q < CW; ++q) lp[q] = 0.f;
             ptx::named_sync(nbar, 128);
-            bool ok = true;
+            // A wait that gives up (timeout or another role's abort) only sets `failed`:
+            // the loop keeps its barrier sequence matched across the warpgroup and the
+            // group leaves together after the item.
+            bool failed = false;
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
                 const int s = (int)(gc & 1);
                 const int pb = (int)(gc % NP);
-                ok = bounded_wait(BAR(C::B_SFULL + s), (uint32_t)((gc >> 1) & 1), abort_flag);
-                ok = ptx::named_red_and(nbar, 128, ok);
-                if (!ok) break;
+                if (!bounded_wait(BAR(C::B_SFULL + s), (uint32_t)((gc >> 1) & 1), abort_flag)) failed = true;
                 ptx::tc_fence_after();
                 if (wg == 0 && t == 0) {
                     // MMA1 of this chunk has finished reading its K slot (and, for the
@@ -602,9 +603,8 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
                     if (c > 0) {
                         // O holds this item's chunks < c: wait for the last of them, rescale our columns
                         const int64_t gp = gc - 1;
-                        ok = bounded_wait(BAR(C::B_ODONE + (int)(gp & 1)), (uint32_t)((gp >> 1) & 1), abort_flag);
-                        ok = ptx::named_red_and(nbar, 128, ok);
-                        if (!ok) break;
+                        if (!bounded_wait(BAR(C::B_ODONE + (int)(gp & 1)), (uint32_t)((gp >> 1) & 1), abort_flag))
+                            failed = true;
                         ptx::tc_fence_after();
 #pragma unroll
                         for (int q0 = 0; q0 < CW; q0 += 8) {
@@ -625,9 +625,8 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
                 // ---- the P buffer is free once the MMA that last read it has completed
                 if (gc >= NP) {
                     const int64_t gr = gc - NP;
-                    ok = bounded_wait(BAR(C::B_ODONE + (int)(gr & 1)), (uint32_t)((gr >> 1) & 1), abort_flag);
-                    ok = ptx::named_red_and(nbar, 128, ok);
-                    if (!ok) break;
+                    if (!bounded_wait(BAR(C::B_ODONE + (int)(gr & 1)), (uint32_t)((gr >> 1) & 1), abort_flag))
+                        failed = true;
                 }
                 // ---- probabilities -> bf16 P^T row of this key, our query columns
                 const uint32_t prow = PBUF(pb);
@@ -657,12 +656,10 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(BAR(C::B_PFULL + pb));
             }
-            if (!ok) break;
             // ===================== epilogue: O / l -> bf16 rows, lse (our query columns)
             const int64_t e = g + nch - 1;
-            ok = bounded_wait(BAR(C::B_ODONE + (int)(e & 1)), (uint32_t)((e >> 1) & 1), abort_flag);
-            ok = ptx::named_red_and(nbar, 128, ok);
-            if (!ok) break;
+            if (!bounded_wait(BAR(C::B_ODONE + (int)(e & 1)), (uint32_t)((e >> 1) & 1), abort_flag)) failed = true;
+            if (ptx::named_red_or(nbar, 128, failed)) break;
             ptx::tc_fence_after();
 #pragma unroll
             for (int q = 0; q < CW; ++q) {
