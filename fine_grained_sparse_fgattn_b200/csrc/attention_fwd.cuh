@@ -131,17 +131,19 @@ struct FwdCfg {
     static constexpr uint32_t AUX_REGS = MQ == 128 ? 80 : 128;
 };
 
-// UMMA shared-memory descriptor (sm_100): start, leading/stride byte offsets,
-// version 1, swizzle mode (2 = 128B, 4 = 64B, 6 = 32B).
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;
-    d |= (uint64_t)layout << 61;
-    return d;
+// UMMA shared-memory descriptor (sm_100): start address >> 4 (bits 0-13), leading
+// byte offset >> 4 (16-29), stride byte offset >> 4 (32-45), version 1 (bit 46),
+// swizzle mode (bits 61-63: 2 = 128B, 4 = 64B, 6 = 32B), built as two halves.  The
+// high half is a compile-time constant per operand; the low half moves by adding
+// (byte offset >> 4), which never carries out of the 14-bit address field for
+// shared-memory offsets below 256 KB.
+__host__ __device__ constexpr uint32_t umma_desc_hi(uint32_t sbo, uint32_t layout) {
+    return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (layout << 29);
 }
+__device__ __forceinline__ uint32_t umma_desc_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t umma_desc_join(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
@@ -442,6 +444,10 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
             constexpr uint32_t IDESC1 = umma_idesc_bf16(128, MQ, false, false);
             constexpr uint32_t IDESC2 = umma_idesc_bf16(D, MQ, true, true);
             constexpr uint32_t P_LAYOUT = (C::P_ROW == 128) ? 2u : (C::P_ROW == 64) ? 4u : 6u;
+            constexpr uint32_t HI_KQ = umma_desc_hi(1024u, 2u);  // K rows and Q rows: K-major, 128B swizzle
+            constexpr uint32_t HI_V = umma_desc_hi(1024u, 2u);   // V^T: MN-major, 128B swizzle
+            constexpr uint32_t HI_P = umma_desc_hi(8u * C::P_ROW, P_LAYOUT);
+            const uint32_t qlo = umma_desc_lo(QTILE, 16u);
             bool ok = true;
             auto issue_pv = [&](int64_t gm, int64_t cm) -> bool {
                 const int vs = (int)(gm % NV);
@@ -450,11 +456,15 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
                 if (!bounded_wait(BAR(C::B_PFULL + pb), (uint32_t)((gm / NP) & 1), abort_flag)) return false;
                 ptx::tc_fence_after();
                 ptx::fence_proxy_async_smem();
-#pragma unroll 1
+                // The descriptors are formed before the MMAs so that the eight issues run
+                // back to back (descriptor arithmetic between issues stalls the single
+                // issuing thread, and with it the tensor pipe).
+                const uint32_t alo = umma_desc_lo(VSLOT(vs), 128u * 128u);
+                const uint32_t blo = umma_desc_lo(PBUF(pb), (uint32_t)C::P_PANEL);
+#pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = umma_desc(VSLOT(vs) + kk * 2048u, 128u * 128u, 1024u, 2u);
-                    const uint64_t bd =
-                        umma_desc(PBUF(pb) + kk * 16u * C::P_ROW, (uint32_t)C::P_PANEL, 8u * C::P_ROW, P_LAYOUT);
+                    const uint64_t ad = umma_desc_join(alo + (uint32_t)(kk * 2048 >> 4), HI_V);
+                    const uint64_t bd = umma_desc_join(blo + (uint32_t)(kk * 16 * C::P_ROW >> 4), HI_P);
                     ptx::mma_bf16_ss(tO, ad, bd, IDESC2, (cm > 0 || kk > 0) ? 1u : 0u);
                 }
                 ptx::mma_commit(BAR(C::B_ODONE + (int)(gm & 1)));
@@ -470,13 +480,15 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
                 if (gc >= 2 && !bounded_wait(BAR(C::B_SFREE + s), (uint32_t)(((gc >> 1) - 1) & 1), abort_flag))
                     return false;
                 ptx::tc_fence_after();
-#pragma unroll 1
+                const uint32_t alo = umma_desc_lo(KSLOT(ks), 16u);
+                const uint32_t dS = tS0 + (uint32_t)s * MQ;
+#pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
                     const uint32_t qoff = (uint32_t)(kk / 4) * (MQ * 128) + (uint32_t)(kk % 4) * 32u;
-                    const uint64_t ad = umma_desc(KSLOT(ks) + koff, 16u, 1024u, 2u);
-                    const uint64_t bd = umma_desc(QTILE + qoff, 16u, 1024u, 2u);
-                    ptx::mma_bf16_ss(tS0 + (uint32_t)s * MQ, ad, bd, IDESC1, kk > 0 ? 1u : 0u);
+                    const uint64_t ad = umma_desc_join(alo + (koff >> 4), HI_KQ);
+                    const uint64_t bd = umma_desc_join(qlo + (qoff >> 4), HI_KQ);
+                    ptx::mma_bf16_ss(dS, ad, bd, IDESC1, kk > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(BAR(C::B_SFULL + s));
                 return true;
