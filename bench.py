@@ -144,7 +144,9 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # traffic figure from the committed ncu summary (valid only for the same kernel source)
 # ---------------------------------------------------------------------------
-def ncu_traffic(workload: str, src_hash: str):
+def ncu_traffic(workload, src_hash: str):
+    if workload is None:
+        return None, None
     path = os.path.join(ROOT, "profiles", f"fgattn_fwd_{workload}.json")
     if not os.path.exists(path):
         return None, None
@@ -212,11 +214,16 @@ def run_reference(args, w):
             secs += sec
             blocks_total += nb
     value = flops_total / secs / 1e12
+    # one step = one whole attention call; the oracle's time for it is extrapolated
+    # from the sample's throughput and the kept work of the sampled heads
+    sample_heads_flops = 4.0 * w.d * float((samp.kept_cnt.reshape(-1, w.QB) * samp.rows[None, :]).sum())
+    call_flops = sample_heads_flops * w.B * w.H / (w.B * samp.H)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * call_flops / (value * 1e12),
+        "ms_per_step_kind": "extrapolated from the sample throughput to one whole attention call",
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": cfg_dict(w, args),
+        "config": cfg_dict(w, args, False),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": samp.cores, "kind": "oracle",
                          "sample": f"{blocks_total} seeded query blocks of heads 0-1 over {args.steps} steps"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -225,10 +232,24 @@ def run_reference(args, w):
     return 0
 
 
-def cfg_dict(w, args):
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 256 * 1024 * 1024
+
+
+def cfg_dict(w, args, flush):
+    l2 = ("L2 flushed before every step (256 MB write, outside the kernel events)" if flush
+          else "inputs larger than L2 (no flush needed)")
     return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "grid": list(w.grid), "d": w.d, "M": w.M, "N": w.N,
             "sparsity_target": w.sparsity, "mask": w.mask, "qkv": w.qkv, "seed": args.seed,
-            "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"heads x{args.gpus} (weak)"}
+            "l2": l2, "parallelism": f"heads x{args.gpus} (weak)",
+            "path": "dense (no kept lists)" if getattr(args, "dense", False) else "tile-sparse (compaction + forward)"}
+
+
+def profile_key(w, args):
+    """Name of the committed ncu summary for this exact workload (None when overridden)."""
+    if args.N is not None or args.sparsity is not None or args.heads is not None or args.dense:
+        return None
+    return w.name
 
 
 # ---------------------------------------------------------------------------
@@ -245,6 +266,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dense", action="store_true",
+                    help="dense run of the same kernel (no kept lists: every key of every block)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.get(args.workload)
@@ -277,18 +300,38 @@ def main():
     lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    def compact():
+        if not args.dense:
+            F.compact_mask(mask, B, H, L, M, N, kept_idx=kept_idx, kept_cnt=kept_cnt, cap=cap)
+
+    def forward():
+        if args.dense:
+            F.forward(q, k, v, None, None, M, N, w.scale, out=out, lse=lse)
+        else:
+            F.forward(q, k, v, kept_idx, kept_cnt, M, N, w.scale, out=out, lse=lse)
+
     def step():
-        F.compact_mask(mask, B, H, L, M, N, kept_idx=kept_idx, kept_cnt=kept_cnt, cap=cap)
-        F.forward(q, k, v, kept_idx, kept_cnt, M, N, w.scale, out=out, lse=lse)
+        compact()
+        forward()
 
     step()
     assert F.device_error() == 0, "device error on the first step"
+    if args.dense:
+        kept_cnt.fill_(L)
     rows = torch.clamp(L - torch.arange(QB, device=dev) * M, max=M).to(torch.float64)
     kept_scores = float((kept_cnt.to(torch.float64) * rows).sum().item())
     flops_per_step = 4.0 * d * kept_scores
     sparsity = 1.0 - kept_scores / (B * H * float(L) * L)
 
+    # Inputs (and the kept lists) smaller than twice the L2 would stay cached between
+    # steps: flush L2 before every step instead, outside the per-kernel events.
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, mask, kept_idx))
+    flush = in_bytes < 2 * L2_BYTES
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
+
     for _ in range(args.warmup):
+        if flush:
+            flush_buf.zero_()
         step()
     torch.cuda.synchronize()
 
@@ -302,11 +345,13 @@ def main():
     with sampler:
         t_start.record(stream)
         for i in range(args.steps):
+            if flush:
+                flush_buf.zero_()
             ev_c[i][0].record(stream)
-            F.compact_mask(mask, B, H, L, M, N, kept_idx=kept_idx, kept_cnt=kept_cnt, cap=cap)
+            compact()
             ev_c[i][1].record(stream)
             ev_f[i][0].record(stream)
-            F.forward(q, k, v, kept_idx, kept_cnt, M, N, w.scale, out=out, lse=lse)
+            forward()
             ev_f[i][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -318,7 +363,8 @@ def main():
     cmp_ms = reduce_max(cmp_ms, dist)
     clocks = sampler.summary()
     assert F.device_error() == 0, "device error in the timed region"
-    ms_per_step = total_ms / args.steps
+    # with a flush between steps the step time is the two kernels' event time
+    ms_per_step = (reduce_max(fwd_ms + cmp_ms, dist) if flush else total_ms / args.steps)
     value = job_throughput(world, flops_per_step, ms_per_step)
 
     # ---- end to end through the public API: pinned host inputs -> device -> host results
@@ -355,10 +401,10 @@ def main():
     peaks, peak_kind = load_peaks()
     achieved = flops_per_step / (fwd_ms * 1e-3) / 1e12
     from fine_grained_sparse_fgattn_b200 import _build
-    traffic, _ = ncu_traffic(w.name, _build.kernel_hash("fwd"))
+    traffic, _ = ncu_traffic(profile_key(w, args), _build.kernel_hash("fwd"))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                "peak_kind": f"{peak_kind} bf16 burst", "kernel": "fgattn_fwd_kernel<128,64>",
+                "peak_kind": f"{peak_kind} bf16 burst", "kernel": f"fgattn_fwd_kernel<{d},{M}>",
                 "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "flops_per_launch": flops_per_step}
 
@@ -373,13 +419,13 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg_dict(w, args),
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg_dict(w, args, flush),
             "forward_ms": fwd_ms, "compact_ms": cmp_ms, "achieved_sparsity": sparsity,
             "pct_of_bf16_peak": 100.0 * value / peaks["bf16_tflops"],
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 2 * args.steps, "clocks": clocks,
+            "gpu_launches": (1 if args.dense else 2) * args.steps, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
