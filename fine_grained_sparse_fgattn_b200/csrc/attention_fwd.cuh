@@ -25,8 +25,9 @@
 // Warp roles (512 threads = four warpgroups):
 //   warps 0-3   softmax warpgroup 0: query columns [0, MQ/2)
 //   warps 4-7   softmax warpgroup 1: query columns [MQ/2, MQ)
-//   warps 8-10  K producer: TMA tile load of the query block; K rows by TMA
-//   warp  11    TMEM allocation + single-thread tcgen05.mma issue
+//   warps 8-9   K producer: TMA tile load of the query block; K rows by TMA
+//   warp  10    single-thread tcgen05.mma issue of the P.V products (MMA2)
+//   warp  11    TMEM allocation + single-thread tcgen05.mma issue of the scores (MMA1)
 //   warps 12-15 V producer: V rows by TMA or cp.async
 // Each chunk is loaded as eight 16-row segments.  A segment whose 16 kept keys
 // are consecutive (always the case for key groups of N >= 16 keys, N a multiple
@@ -116,7 +117,7 @@ struct FwdCfg {
     static constexpr int B_KFULL = 0, B_KEMPTY = NK, B_VFULL = 2 * NK, B_VEMPTY = 2 * NK + NV;
     static constexpr int B_QFULL = 2 * NK + 2 * NV, B_QEMPTY = B_QFULL + 1, B_SFULL = B_QFULL + 2;
     static constexpr int B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_ODONE = B_PFULL + NP;
-    static constexpr int B_DRAIN = B_ODONE + 2, NBAR = B_DRAIN + 1;
+    static constexpr int B_DRAIN = B_ODONE + 2, B_DRAIN2 = B_DRAIN + 1, NBAR = B_DRAIN2 + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
     static constexpr int BYTES = OFF_ABORT + 8;
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < NK; ++i) {
-            ptx::mbar_init(BAR(C::B_KFULL + i), 3);
+            ptx::mbar_init(BAR(C::B_KFULL + i), 2);
             ptx::mbar_init(BAR(C::B_KEMPTY + i), 1);
         }
         for (int i = 0; i < NV; ++i) {
@@ -263,6 +264,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
         }
         for (int i = 0; i < NP; ++i) ptx::mbar_init(BAR(C::B_PFULL + i), 256);
         ptx::mbar_init(BAR(C::B_DRAIN), 1);
+        ptx::mbar_init(BAR(C::B_DRAIN2), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -274,13 +276,13 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
     const uint32_t tO = tmem + 2u * MQ;  // O^T accumulator: columns [2MQ, 3MQ)
     const int64_t L = p.L;
 
-    if (warp >= 8 && warp < 11) {
+    if (warp >= 8 && warp < 10) {
         // ===================================================== K producer (TMA)
         if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
         const int kw = warp - 8;
-        // segments 0-2 -> warp 8, 3-5 -> warp 9, 6-7 -> warp 10; four lanes (4-row groups) each
-        const int seg0 = kw * 3;
-        const int nseg = kw < 2 ? 3 : 2;
+        // segments 0-3 -> warp 8, 4-7 -> warp 9; four lanes (4-row groups) each
+        const int seg0 = kw * 4;
+        const int nseg = 4;
         const int g4 = seg0 * 4 + lane;            // this lane's 4-row group in the chunk
         const bool issuer = lane < nseg * 4;
         const int lseg = lane >> 2;                // segment within the warp
@@ -437,8 +439,13 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
             g += nch;
         }
         ptx::cp_async_wait_all();
-    } else if (warp == 11) {
-        // ===================================================== MMA issuer
+    } else if (warp == 10 || warp == 11) {
+        // ===================================================== MMA issuers
+        // Two issuing threads, one per MMA kind, so that neither waits behind the
+        // other's inputs: warp 11 issues the scores of a chunk as soon as its K rows
+        // have landed and its TMEM slot is free; warp 10 issues the P.V of a chunk as
+        // soon as its V rows and probabilities are ready.  The tensor pipe takes the
+        // two streams in arrival order; each thread's commits track its own MMAs.
         if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
         if (lane == 0) {
             constexpr uint32_t IDESC1 = umma_idesc_bf16(128, MQ, false, false);
@@ -493,23 +500,16 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
                 ptx::mma_commit(BAR(C::B_SFULL + s));
                 return true;
             };
-            // Issue order within an item: S of chunks 0 and 1, then for every chunk c
-            // the S of chunk c+2 (as soon as its slot frees, early in softmax(c)) before
-            // the P.V of chunk c (which waits for the end of softmax(c)).  The tensor core
-            // thus computes the next scores while the softmax works on the current ones.
             int64_t g = 0, it = 0;
             for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
                 const int64_t nch = (item_count(p, item, false) + 127) / 128;
-                for (int64_t c = 0; c < nch && c < 2 && ok; ++c) ok = issue_s(g + c, c, it);
-                for (int64_t c = 0; c < nch && ok; ++c) {
-                    if (c + 2 < nch) ok = issue_s(g + c + 2, c + 2, it);
-                    if (ok) ok = issue_pv(g + c, c);
-                }
+                for (int64_t c = 0; c < nch && ok; ++c) ok = (warp == 11) ? issue_s(g + c, c, it) : issue_pv(g + c, c);
                 g += nch;
             }
             // drain: every MMA this thread issued has completed before TMEM is freed
-            ptx::mma_commit(BAR(C::B_DRAIN));
-            bounded_wait(BAR(C::B_DRAIN), 0u, abort_flag, /*honour_abort=*/false);
+            const int drain = (warp == 11) ? C::B_DRAIN : C::B_DRAIN2;
+            ptx::mma_commit(BAR(drain));
+            bounded_wait(BAR(drain), 0u, abort_flag, /*honour_abort=*/false);
         }
         __syncwarp();
     } else {
