@@ -13,8 +13,9 @@
 //     O^T [D x MQ]        += V_chunk^T [D x 128] . P^T [128 x MQ]  (MMA2, M=D)
 // Putting the gathered keys on the MMA's M dimension keeps every MMA at the
 // full-rate M=128 shape for any query-block height MQ in {16, 32, 64, 128}.
-// A softmax thread owns one key (TMEM lane) of the chunk; two softmax
-// warpgroups split the chunk's MQ query columns between them.  The per-query
+// A softmax thread owns one key (TMEM lane) of the chunk; the softmax
+// warpgroups split the chunk's MQ query columns between them (more groups =
+// shorter per-thread dependency chains per chunk).  The per-query
 // running maximum is a cross-lane quantity, so it is refreshed lazily:
 // probabilities are taken against a per-query reference mref, and only when a
 // score exceeds mref by more than TAU (log2 units) is the reference raised and
@@ -22,13 +23,13 @@
 // uses the same reference, so the result is exact up to rounding whatever
 // reference was used.
 //
-// Warp roles (512 threads = four warpgroups):
-//   warps 0-3   softmax warpgroup 0: query columns [0, MQ/2)
-//   warps 4-7   softmax warpgroup 1: query columns [MQ/2, MQ)
-//   warps 8-9   K producer: TMA tile load of the query block; K rows by TMA
-//   warp  10    single-thread tcgen05.mma issue of the P.V products (MMA2)
-//   warp  11    TMEM allocation + single-thread tcgen05.mma issue of the scores (MMA1)
-//   warps 12-15 V producer: V rows by TMA or cp.async
+// Warp roles (NSW softmax warpgroups + two auxiliary warpgroups; NSW = 4, 768
+// threads, for MQ in {32, 64}; NSW = 2, 512 threads, for MQ in {16, 128}):
+//   warps 0 .. 4*NSW-1  softmax warpgroup g: query columns [g*CW, (g+1)*CW), CW = MQ/NSW
+//   warps A, A+1        K producer (A = 4*NSW): TMA tile load of the query block; K rows by TMA
+//   warp  A+2           single-thread tcgen05.mma issue of the P.V products (MMA2)
+//   warp  A+3           TMEM allocation + single-thread tcgen05.mma issue of the scores (MMA1)
+//   warps A+4 .. A+7    V producer: V rows by TMA or cp.async
 // Each chunk is loaded as eight 16-row segments.  A segment whose 16 kept keys
 // are consecutive (always the case for key groups of N >= 16 keys, N a multiple
 // of 16) is one tiled TMA box; any other segment is gathered row by row (K with
@@ -78,19 +79,20 @@ struct FwdCfg {
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(MQ == 16 || MQ == 32 || MQ == 64 || MQ == 128, "query block");
     static constexpr int KC = 128;              // keys per chunk = MMA1 M
-    static constexpr int CW = MQ / 2;           // query columns per softmax warpgroup
+    static constexpr int NSW = (MQ == 32 || MQ == 64) ? 4 : 2;  // softmax warpgroups
+    static constexpr int CW = MQ / NSW;         // query columns per softmax warpgroup
     static constexpr int KV_TILE = KC * D * 2;  // bytes of a K or V chunk
     static constexpr int P_ROW = (MQ * 2 < 128) ? MQ * 2 : 128;  // bytes per key row of a P panel
     static constexpr int P_CPR = P_ROW / 16;    // 16-byte chunks per P row
     static constexpr int P_PANEL = KC * P_ROW;  // bytes per P panel
     static constexpr int P_TILE = KC * MQ * 2;
     static constexpr int Q_TILE = MQ * D * 2;
-    static constexpr int SROWS = (CW < 16) ? CW : 16;  // epilogue staging rows per warpgroup
+    static constexpr int SROWS = (CW < 8) ? CW : (NSW == 4 ? 8 : (CW < 16 ? CW : 16));  // staging rows per group
     static constexpr int STAGE = SROWS * D * 2;
-    static constexpr int MISC = 2 * (3 * CW + 4 * CW) * 4 + 64 * 8 + 64;  // mref/alpha/lfin/red, barriers
+    static constexpr int MISC = NSW * (3 * CW + 4 * CW) * 4 + 64 * 8 + 64;  // mref/alpha/lfin/red, barriers
     static constexpr int LIMIT = 227 * 1024 - 1024 - 256;
     static constexpr int fixed_bytes(int nk, int nv, int np) {
-        return nk * KV_TILE + nv * KV_TILE + np * P_TILE + Q_TILE + 2 * STAGE + MISC;
+        return nk * KV_TILE + nv * KV_TILE + np * P_TILE + Q_TILE + NSW * STAGE + MISC;
     }
     // pipeline depths: K ring, V ring, P buffers (deepest that fits)
     // The V ring has two stages so that "V slot free" is exactly "MMA2 of the chunk
@@ -103,12 +105,12 @@ struct FwdCfg {
     static constexpr int OFF_V = OFF_K + NK * KV_TILE;
     static constexpr int OFF_P = OFF_V + NV * KV_TILE;
     static constexpr int OFF_Q = OFF_P + NP * P_TILE;
-    static constexpr int OFF_STAGE = OFF_Q + Q_TILE;         // 2 x STAGE
-    static constexpr int OFF_MREF = OFF_STAGE + 2 * STAGE;   // [2][CW]
-    static constexpr int OFF_ALPHA = OFF_MREF + 2 * CW * 4;  // [2][CW]
-    static constexpr int OFF_LFIN = OFF_ALPHA + 2 * CW * 4;  // [2][CW]
-    static constexpr int OFF_RED = OFF_LFIN + 2 * CW * 4;    // [2][4][CW]
-    static constexpr int OFF_BAR = (OFF_RED + 2 * 4 * CW * 4 + 7) / 8 * 8;
+    static constexpr int OFF_STAGE = OFF_Q + Q_TILE;           // NSW x STAGE
+    static constexpr int OFF_MREF = OFF_STAGE + NSW * STAGE;   // [NSW][CW]
+    static constexpr int OFF_ALPHA = OFF_MREF + NSW * CW * 4;  // [NSW][CW]
+    static constexpr int OFF_LFIN = OFF_ALPHA + NSW * CW * 4;  // [NSW][CW]
+    static constexpr int OFF_RED = OFF_LFIN + NSW * CW * 4;    // [NSW][4][CW]
+    static constexpr int OFF_BAR = (OFF_RED + NSW * 4 * CW * 4 + 7) / 8 * 8;
     // barriers: k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] (unused: o_done serves) q_full q_empty
     //           s_full[2] s_free[2] p_full[NP] o_done[2] drain
     // Only s_full and o_done are tensor-core commits (each commit costs tensor-pipe
@@ -124,12 +126,18 @@ struct FwdCfg {
     static_assert(BYTES <= LIMIT, "shared memory layout");
     static constexpr int SMEM_REQUEST = BYTES + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = (3 * MQ <= 64) ? 64 : (3 * MQ <= 128) ? 128 : (3 * MQ <= 256) ? 256 : 512;
-    static constexpr int THREADS = 512;
-    // Register split between the two softmax warpgroups and the two producer/MMA
-    // warpgroups (2*128*SOFT + 2*128*AUX = 512*128).  MQ = 128 keeps 64 columns of
-    // scores and sums per softmax thread and needs the larger share.
-    static constexpr uint32_t SOFT_REGS = MQ == 128 ? 176 : 128;
-    static constexpr uint32_t AUX_REGS = MQ == 128 ? 80 : 128;
+    static constexpr int SOFT_THREADS = 128 * NSW;
+    static constexpr int THREADS = SOFT_THREADS + 256;
+    static constexpr int AUX_WARP = 4 * NSW;  // first auxiliary warp
+    // Register split between the softmax warpgroups and the two producer/MMA
+    // warpgroups; it must add up to the launch's allocation (THREADS x the per-thread
+    // count the launch bounds give: 128 at 512 threads, 80 at 768):
+    //   NSW = 2: 2*128*SOFT + 2*128*AUX = 512*128;  NSW = 4: 4*128*88 + 2*128*64 = 768*80.
+    // MQ = 128 keeps 64 columns of scores and sums per softmax thread.
+    static constexpr uint32_t LAUNCH_REGS = NSW == 4 ? 80 : 128;
+    static constexpr uint32_t SOFT_REGS = NSW == 4 ? 88 : (MQ == 128 ? 176 : 128);
+    static constexpr uint32_t AUX_REGS = NSW == 4 ? 64 : (MQ == 128 ? 80 : 128);
+    static_assert(NSW * 128 * SOFT_REGS + 256 * AUX_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
 // UMMA shared-memory descriptor (sm_100): start address >> 4 (bits 0-13), leading
@@ -223,7 +231,7 @@ __device__ __forceinline__ void rows_of(const FwdParams& p, int4 raw, int64_t ro
 }
 
 template <int D, int MQ>
-__global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = FwdCfg<D, MQ>;
     constexpr int NK = C::NK, NV = C::NV, NP = C::NP, CW = C::CW;
     constexpr float TAU = 8.0f;
@@ -241,8 +249,9 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    constexpr int AW = C::AUX_WARP;
 
-    if (warp == 11) {
+    if (warp == AW + 3) {
         ptx::tmem_alloc(sbase + C::OFF_TMEM, C::TMEM_COLS);
         ptx::tmem_relinquish();
     }
@@ -259,10 +268,10 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
         ptx::mbar_init(BAR(C::B_QEMPTY), 1);
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(BAR(C::B_SFULL + i), 1);
-            ptx::mbar_init(BAR(C::B_SFREE + i), 256);
+            ptx::mbar_init(BAR(C::B_SFREE + i), C::SOFT_THREADS);
             ptx::mbar_init(BAR(C::B_ODONE + i), 1);
         }
-        for (int i = 0; i < NP; ++i) ptx::mbar_init(BAR(C::B_PFULL + i), 256);
+        for (int i = 0; i < NP; ++i) ptx::mbar_init(BAR(C::B_PFULL + i), C::SOFT_THREADS);
         ptx::mbar_init(BAR(C::B_DRAIN), 1);
         ptx::mbar_init(BAR(C::B_DRAIN2), 1);
         *abort_flag = 0;
@@ -276,11 +285,11 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
     const uint32_t tO = tmem + 2u * MQ;  // O^T accumulator: columns [2MQ, 3MQ)
     const int64_t L = p.L;
 
-    if (warp >= 8 && warp < 10) {
+    if (warp >= AW && warp < AW + 2) {
         // ===================================================== K producer (TMA)
-        if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
-        const int kw = warp - 8;
-        // segments 0-3 -> warp 8, 4-7 -> warp 9; four lanes (4-row groups) each
+        if constexpr (C::AUX_REGS != C::LAUNCH_REGS) ptx::regs_dec<C::AUX_REGS>();
+        const int kw = warp - AW;
+        // segments 0-3 -> first warp, 4-7 -> second; four lanes (4-row groups) each
         const int seg0 = kw * 4;
         const int nseg = 4;
         const int g4 = seg0 * 4 + lane;            // this lane's 4-row group in the chunk
@@ -288,15 +297,15 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
         const int lseg = lane >> 2;                // segment within the warp
         int64_t g = 0, it = 0;
         int64_t issued = 0;    // chunks whose loads this warp has issued
-        int64_t q_issued = 0;  // query tiles issued (warp 8)
+        int64_t q_issued = 0;  // query tiles issued (first K warp)
         bool ok = true;
         for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
             const int64_t bh = item / p.QB;
             const int64_t qb = item - bh * p.QB;
-            const int64_t cnt = item_count(p, item, warp == 8 && lane == 0);
+            const int64_t cnt = item_count(p, item, kw == 0 && lane == 0);
             const int64_t nch = (cnt + 127) / 128;
             const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
-            if (warp == 8) {  // the query tile (rows past L are padding; their results are never stored)
+            if (kw == 0) {  // the query tile (rows past L are padding; their results are never stored)
                 const bool okq = it == 0 || bounded_wait(BAR(C::B_QEMPTY), (uint32_t)((it - 1) & 1), abort_flag);
                 if (!__all_sync(0xffffffffu, okq)) {
                     ok = false;
@@ -367,10 +376,10 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
         for (int64_t i = issued > NK ? issued - NK : 0; i < issued; ++i)
             bounded_wait(BAR(C::B_KFULL + (int)(i % NK)), (uint32_t)((i / NK) & 1), abort_flag, false);
         if (q_issued > 0) bounded_wait(BAR(C::B_QFULL), (uint32_t)((q_issued - 1) & 1), abort_flag, false);
-    } else if (warp >= 12) {
+    } else if (warp >= AW + 4) {
         // ===================================================== V producer (TMA boxes / cp.async)
-        if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
-        const int vw = warp - 12;      // rows [32*vw, 32*vw + 32) of each chunk = two segments
+        if constexpr (C::AUX_REGS != C::LAUNCH_REGS) ptx::regs_dec<C::AUX_REGS>();
+        const int vw = warp - (AW + 4);  // rows [32*vw, 32*vw + 32) of each chunk = two segments
         constexpr int PPR = D / 8;     // 16-byte pieces per row
         constexpr int RPI = 32 / PPR;  // rows per warp instruction
         int64_t g = 0;
@@ -439,14 +448,14 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
             g += nch;
         }
         ptx::cp_async_wait_all();
-    } else if (warp == 10 || warp == 11) {
+    } else if (warp == AW + 2 || warp == AW + 3) {
         // ===================================================== MMA issuers
         // Two issuing threads, one per MMA kind, so that neither waits behind the
-        // other's inputs: warp 11 issues the scores of a chunk as soon as its K rows
-        // have landed and its TMEM slot is free; warp 10 issues the P.V of a chunk as
+        // other's inputs: warp A+3 issues the scores of a chunk as soon as its K rows
+        // have landed and its TMEM slot is free; warp A+2 issues the P.V of a chunk as
         // soon as its V rows and probabilities are ready.  The tensor pipe takes the
         // two streams in arrival order; each thread's commits track its own MMAs.
-        if constexpr (C::AUX_REGS != 128) ptx::regs_dec<C::AUX_REGS>();
+        if constexpr (C::AUX_REGS != C::LAUNCH_REGS) ptx::regs_dec<C::AUX_REGS>();
         if (lane == 0) {
             constexpr uint32_t IDESC1 = umma_idesc_bf16(128, MQ, false, false);
             constexpr uint32_t IDESC2 = umma_idesc_bf16(D, MQ, true, true);
@@ -503,19 +512,19 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
             int64_t g = 0, it = 0;
             for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
                 const int64_t nch = (item_count(p, item, false) + 127) / 128;
-                for (int64_t c = 0; c < nch && ok; ++c) ok = (warp == 11) ? issue_s(g + c, c, it) : issue_pv(g + c, c);
+                for (int64_t c = 0; c < nch && ok; ++c) ok = (warp == AW + 3) ? issue_s(g + c, c, it) : issue_pv(g + c, c);
                 g += nch;
             }
             // drain: every MMA this thread issued has completed before TMEM is freed
-            const int drain = (warp == 11) ? C::B_DRAIN : C::B_DRAIN2;
+            const int drain = (warp == AW + 3) ? C::B_DRAIN : C::B_DRAIN2;
             ptx::mma_commit(BAR(drain));
             bounded_wait(BAR(drain), 0u, abort_flag, /*honour_abort=*/false);
         }
         __syncwarp();
     } else {
-        // ===================================================== softmax / epilogue (two warpgroups)
-        if constexpr (C::SOFT_REGS != 128) ptx::regs_inc<C::SOFT_REGS>();
-        const int wg = warp >> 2;         // 0 or 1
+        // ===================================================== softmax / epilogue (NSW warpgroups)
+        if constexpr (C::SOFT_REGS != C::LAUNCH_REGS) ptx::regs_inc<C::SOFT_REGS>();
+        const int wg = warp >> 2;         // 0 .. NSW-1
         const int wq = warp & 3;          // warp within the group = TMEM lane quarter
         const int t = threadIdx.x & 127;  // key lane within a chunk; TMEM lane t
         const uint32_t nbar = 1u + (uint32_t)wg;
@@ -726,7 +735,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_kernel(const __grid_constan
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (warp == 11) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == AW + 3) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace fgattn

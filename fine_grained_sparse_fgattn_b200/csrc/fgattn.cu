@@ -69,6 +69,13 @@ fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const void* k, c
         if (cudaFuncSetAttribute(fgattn::fgattn_fwd_kernel<D, MQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem) != cudaSuccess)
             return FGATTN_ERR_CUDA;
+        // The warp roles re-divide the block's registers with setmaxnreg, which only
+        // completes if the launch allocates exactly the per-thread count the split
+        // was sized for: refuse to launch otherwise (it would wait forever).
+        cudaFuncAttributes attr;
+        if (cudaFuncGetAttributes(&attr, fgattn::fgattn_fwd_kernel<D, MQ>) != cudaSuccess) return FGATTN_ERR_CUDA;
+        const bool split = C::SOFT_REGS != C::LAUNCH_REGS || C::AUX_REGS != C::LAUNCH_REGS;
+        if (split && attr.numRegs != (int)C::LAUNCH_REGS) return FGATTN_ERR_UNSUPPORTED;
         configured = true;
     }
     const int sms = current_sms();
