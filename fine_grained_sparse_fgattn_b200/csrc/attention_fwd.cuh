@@ -133,6 +133,8 @@ struct FwdCfg {
     // warpgroups; it must add up to the launch's allocation (THREADS x the per-thread
     // count the launch bounds give: 128 at 512 threads, 80 at 768):
     //   NSW = 2: 2*128*SOFT + 2*128*AUX = 512*128;  NSW = 4: 4*128*88 + 2*128*64 = 768*80.
+    // (The producer and issuer warps fit in 64 registers at NSW = 4; at MQ = 128 they
+    // keep 80, which measured faster than a 192/64 split.)
     // MQ = 128 keeps 64 columns of scores and sums per softmax thread.
     static constexpr uint32_t LAUNCH_REGS = NSW == 4 ? 80 : 128;
     static constexpr uint32_t SOFT_REGS = NSW == 4 ? 88 : (MQ == 128 ? 176 : 128);
@@ -553,59 +555,71 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(c
             // the loop keeps its barrier sequence matched across the warpgroup and the
             // group leaves together after the item.
             bool failed = false;
-            for (int64_t c = 0; c < nch; ++c) {
-                const int64_t gc = g + c;
-                const int s = (int)(gc & 1);
-                const int pb = (int)(gc % NP);
-                if (!bounded_wait(BAR(C::B_SFULL + s), (uint32_t)((gc >> 1) & 1), abort_flag)) failed = true;
+            float v[CW];
+            // Wait for the scores of item chunk cc, release what their MMA read, and load
+            // them into dst.
+            auto load_chunk = [&](int64_t cc, auto& dst) {
+                const int64_t gx = g + cc;
+                const int sx = (int)(gx & 1);
+                if (!bounded_wait(BAR(C::B_SFULL + sx), (uint32_t)((gx >> 1) & 1), abort_flag)) failed = true;
                 ptx::tc_fence_after();
                 if (wg == 0 && t == 0) {
                     // MMA1 of this chunk has finished reading its K slot (and, for the
                     // item's last chunk, the query tile)
-                    ptx::mbar_arrive(BAR(C::B_KEMPTY + (int)(gc % NK)));
-                    if (c == nch - 1) ptx::mbar_arrive(BAR(C::B_QEMPTY));
+                    ptx::mbar_arrive(BAR(C::B_KEMPTY + (int)(gx % NK)));
+                    if (cc == nch - 1) ptx::mbar_arrive(BAR(C::B_QEMPTY));
                 }
-                float v[CW];
-                {
-                    const uint32_t ta = tS0 + (uint32_t)s * MQ + col0 + lane_base;
-                    if constexpr (CW >= 32) {
+                const uint32_t ta = tS0 + (uint32_t)sx * MQ + col0 + lane_base;
+                if constexpr (CW >= 32) {
 #pragma unroll
-                        for (int pi = 0; pi < CW / 32; ++pi) {
-                            float tmp[32];
-                            ptx::tmem_ld32(ta + pi * 32, tmp);
+                    for (int pi = 0; pi < CW / 32; ++pi) {
+                        float tmp[32];
+                        ptx::tmem_ld32(ta + pi * 32, tmp);
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) v[pi * 32 + j] = tmp[j];
-                        }
-                    } else if constexpr (CW == 16) {
-                        float tmp[16];
-                        ptx::tmem_ld16(ta, tmp);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) v[j] = tmp[j];
-                    } else {
-                        float tmp[8];
-                        ptx::tmem_ld8(ta, tmp);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) v[j] = tmp[j];
+                        for (int j = 0; j < 32; ++j) dst[pi * 32 + j] = tmp[j];
                     }
-                    ptx::tmem_wait_ld();
+                } else if constexpr (CW == 16) {
+                    ptx::tmem_ld16(ta, dst);
+                } else {
+                    ptx::tmem_ld8(ta, dst);
                 }
+            };
+            load_chunk(0, v);
+            for (int64_t c = 0; c < nch; ++c) {
+                const int64_t gc = g + c;
+                const int s = (int)(gc & 1);
+                const int pb = (int)(gc % NP);
+                if (c > 0) load_chunk(c, v);
+                ptx::tmem_wait_ld();
+                // the scores are in registers: the slot is free for the MMA of chunk gc+2
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(BAR(C::B_SFREE + s));
                 const bool valid = c * 128 + t < cnt;
-                // ---- largest excess of this key's scores over the references (log2 units)
-                float dmax = -INFINITY;
+                // ---- v <- score * scale * log2(e) - reference, and the largest excess over
+                // the references (log2 units).  The first chunk of an item always takes the
+                // exact path below (the references start at -inf).
+                bool need = true;
+                if (c > 0) {
+                    float dmax = -INFINITY;
 #pragma unroll
-                for (int q = 0; q < CW; q += 4) {
-                    const float4 m4 = *reinterpret_cast<const float4*>(mref + q);
-                    dmax = ptx::max3(dmax, fmaf(v[q], cs, -m4.x), fmaf(v[q + 1], cs, -m4.y));
-                    dmax = ptx::max3(dmax, fmaf(v[q + 2], cs, -m4.z), fmaf(v[q + 3], cs, -m4.w));
+                    for (int q = 0; q < CW; q += 4) {
+                        const float4 m4 = *reinterpret_cast<const float4*>(mref + q);
+                        v[q] = fmaf(v[q], cs, -m4.x);
+                        v[q + 1] = fmaf(v[q + 1], cs, -m4.y);
+                        v[q + 2] = fmaf(v[q + 2], cs, -m4.z);
+                        v[q + 3] = fmaf(v[q + 3], cs, -m4.w);
+                        dmax = ptx::max3(dmax, v[q], v[q + 1]);
+                        dmax = ptx::max3(dmax, v[q + 2], v[q + 3]);
+                    }
+                    need = ptx::named_red_or(nbar, 128, valid && dmax > TAU);
                 }
-                const bool need = ptx::named_red_or(nbar, 128, valid && dmax > TAU);
                 if (need) {
-                    // ---- exact column maxima of this chunk -> raised references
+                    // ---- back to scaled scores, exact column maxima -> raised references
+#pragma unroll
+                    for (int q = 0; q < CW; ++q) v[q] = (c == 0) ? v[q] * cs : v[q] + mref[q];
 #pragma unroll
                     for (int q = 0; q < CW; ++q) {
-                        float x = valid ? v[q] * cs : -INFINITY;
+                        float x = valid ? v[q] : -INFINITY;
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
                         if (lane == (q & 31)) red[wq * CW + q] = x;
@@ -620,7 +634,10 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(c
                     }
                     ptx::named_sync(nbar, 128);
 #pragma unroll
-                    for (int q = 0; q < CW; ++q) lp[q] *= alpha[q];
+                    for (int q = 0; q < CW; ++q) {
+                        lp[q] *= alpha[q];
+                        v[q] -= mref[q];
+                    }
                     if (c > 0) {
                         // O holds this item's chunks < c: wait for the last of them, rescale our columns
                         const int64_t gp = gc - 1;
@@ -637,6 +654,8 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(c
                             ptx::tmem_st8(tO + col0 + q0 + lane_base, o);
                         }
                         ptx::tmem_wait_st();
+                        // the rescaled accumulator must reach TMEM before the next P.V
+                        ptx::tc_fence_before();
                     }
                 }
                 if (!valid) {
@@ -653,14 +672,11 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(c
                 const uint32_t prow = PBUF(pb);
 #pragma unroll
                 for (int q = 0; q < CW; q += 8) {
-                    const float4 ma = *reinterpret_cast<const float4*>(mref + q);
-                    const float4 mb = *reinterpret_cast<const float4*>(mref + q + 4);
-                    const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
                     uint32_t packed[4];
 #pragma unroll
                     for (int j = 0; j < 8; j += 2) {
-                        const float p0 = ptx::ex2(fmaf(v[q + j], cs, -mm[j]));
-                        const float p1 = ptx::ex2(fmaf(v[q + j + 1], cs, -mm[j + 1]));
+                        const float p0 = ptx::ex2(v[q + j]);
+                        const float p1 = ptx::ex2(v[q + j + 1]);
                         lp[q + j] += p0;
                         lp[q + j + 1] += p1;
                         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
@@ -673,8 +689,8 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(c
                                  "r"(packed[1]), "r"(packed[2]), "r"(packed[3])
                                  : "memory");
                 }
+                // generic-proxy P writes -> visible to the tensor core's async proxy
                 ptx::fence_proxy_async_smem();
-                ptx::tc_fence_before();
                 ptx::mbar_arrive(BAR(C::B_PFULL + pb));
             }
             // ===================== epilogue: O / l -> bf16 rows, lse (our query columns)
