@@ -23,13 +23,18 @@
 // uses the same reference, so the result is exact up to rounding whatever
 // reference was used.
 //
-// Warp roles (NSW softmax warpgroups + two auxiliary warpgroups; NSW = 4, 768
-// threads, for MQ in {32, 64}; NSW = 2, 512 threads, for MQ in {16, 128}):
+// Two warp layouts (template parameter GATHER), each the faster one for its kind
+// of key list.  Tile layout (lists made of 16-key runs: N a multiple of 16, or a
+// dense run): NSW softmax warpgroups (4, i.e. 768 threads, for MQ in {32, 64}; 2
+// otherwise) + two auxiliary warpgroups:
 //   warps 0 .. 4*NSW-1  softmax warpgroup g: query columns [g*CW, (g+1)*CW), CW = MQ/NSW
 //   warps A, A+1        K producer (A = 4*NSW): TMA tile load of the query block; K rows by TMA
 //   warp  A+2           single-thread tcgen05.mma issue of the P.V products (MMA2)
 //   warp  A+3           TMEM allocation + single-thread tcgen05.mma issue of the scores (MMA1)
 //   warps A+4 .. A+7    V producer: V rows by TMA or cp.async
+// Gather layout (other lists: rows fetched one by one, where issuing the K row
+// gathers dominates): two softmax warpgroups (512 threads), three K producer warps
+// (A .. A+2) and one warp (A+3) issuing both MMA kinds, scores two chunks ahead.
 // Each chunk is loaded as eight 16-row segments.  A segment whose 16 kept keys
 // are consecutive (always the case for key groups of N >= 16 keys, N a multiple
 // of 16) is one tiled TMA box; any other segment is gathered row by row (K with
@@ -74,12 +79,13 @@ struct alignas(64) FwdParams {
     float scale_log2;  // scale * log2(e)
 };
 
-template <int D, int MQ>
+template <int D, int MQ, bool GATHER>
 struct FwdCfg {
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(MQ == 16 || MQ == 32 || MQ == 64 || MQ == 128, "query block");
     static constexpr int KC = 128;              // keys per chunk = MMA1 M
-    static constexpr int NSW = (MQ == 32 || MQ == 64) ? 4 : 2;  // softmax warpgroups
+    static constexpr int NSW = (!GATHER && (MQ == 32 || MQ == 64)) ? 4 : 2;  // softmax warpgroups
+    static constexpr int KWARPS = GATHER ? 3 : 2;                            // K producer warps
     static constexpr int CW = MQ / NSW;         // query columns per softmax warpgroup
     static constexpr int KV_TILE = KC * D * 2;  // bytes of a K or V chunk
     static constexpr int P_ROW = (MQ * 2 < 128) ? MQ * 2 : 128;  // bytes per key row of a P panel
@@ -232,9 +238,10 @@ __device__ __forceinline__ void rows_of(const FwdParams& p, int4 raw, int64_t ro
     }
 }
 
-template <int D, int MQ>
-__global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(const __grid_constant__ FwdParams p) {
-    using C = FwdCfg<D, MQ>;
+template <int D, int MQ, bool GATHER>
+__global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
+    fgattn_fwd_kernel(const __grid_constant__ FwdParams p) {
+    using C = FwdCfg<D, MQ, GATHER>;
     constexpr int NK = C::NK, NV = C::NV, NP = C::NP, CW = C::CW;
     constexpr float TAU = 8.0f;
 
@@ -259,7 +266,7 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(c
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < NK; ++i) {
-            ptx::mbar_init(BAR(C::B_KFULL + i), 2);
+            ptx::mbar_init(BAR(C::B_KFULL + i), C::KWARPS);
             ptx::mbar_init(BAR(C::B_KEMPTY + i), 1);
         }
         for (int i = 0; i < NV; ++i) {
@@ -287,13 +294,14 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(c
     const uint32_t tO = tmem + 2u * MQ;  // O^T accumulator: columns [2MQ, 3MQ)
     const int64_t L = p.L;
 
-    if (warp >= AW && warp < AW + 2) {
+    if (warp >= AW && warp < AW + C::KWARPS) {
         // ===================================================== K producer (TMA)
         if constexpr (C::AUX_REGS != C::LAUNCH_REGS) ptx::regs_dec<C::AUX_REGS>();
         const int kw = warp - AW;
-        // segments 0-3 -> first warp, 4-7 -> second; four lanes (4-row groups) each
-        const int seg0 = kw * 4;
-        const int nseg = 4;
+        // tile layout: segments 0-3 -> first warp, 4-7 -> second; gather layout: 0-2, 3-5, 6-7;
+        // four lanes (4-row groups) per segment
+        const int seg0 = GATHER ? kw * 3 : kw * 4;
+        const int nseg = GATHER ? (kw < 2 ? 3 : 2) : 4;
         const int g4 = seg0 * 4 + lane;            // this lane's 4-row group in the chunk
         const bool issuer = lane < nseg * 4;
         const int lseg = lane >> 2;                // segment within the warp
@@ -450,7 +458,7 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(c
             g += nch;
         }
         ptx::cp_async_wait_all();
-    } else if (warp == AW + 2 || warp == AW + 3) {
+    } else if (warp == AW + 3 || (!GATHER && warp == AW + 2)) {
         // ===================================================== MMA issuers
         // Two issuing threads, one per MMA kind, so that neither waits behind the
         // other's inputs: warp A+3 issues the scores of a chunk as soon as its K rows
@@ -514,7 +522,18 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ>::THREADS, 1) fgattn_fwd_kernel(c
             int64_t g = 0, it = 0;
             for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
                 const int64_t nch = (item_count(p, item, false) + 127) / 128;
-                for (int64_t c = 0; c < nch && ok; ++c) ok = (warp == AW + 3) ? issue_s(g + c, c, it) : issue_pv(g + c, c);
+                if constexpr (GATHER) {
+                    // one issuing thread: S of chunks 0 and 1, then for every chunk c the
+                    // S of chunk c+2 (its slot frees early in softmax(c)) before the P.V of c
+                    for (int64_t c = 0; c < nch && c < 2 && ok; ++c) ok = issue_s(g + c, c, it);
+                    for (int64_t c = 0; c < nch && ok; ++c) {
+                        if (c + 2 < nch) ok = issue_s(g + c + 2, c + 2, it);
+                        if (ok) ok = issue_pv(g + c, c);
+                    }
+                } else {
+                    for (int64_t c = 0; c < nch && ok; ++c)
+                        ok = (warp == AW + 3) ? issue_s(g + c, c, it) : issue_pv(g + c, c);
+                }
                 g += nch;
             }
             // drain: every MMA this thread issued has completed before TMEM is freed

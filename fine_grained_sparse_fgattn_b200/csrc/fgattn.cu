@@ -53,10 +53,10 @@ int current_sms() {
     return sms;
 }
 
-template <int D, int MQ>
+template <int D, int MQ, bool GATHER>
 fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const void* k, const void* v, int64_t rows,
                          cudaStream_t stream) {
-    using C = fgattn::FwdCfg<D, MQ>;
+    using C = fgattn::FwdCfg<D, MQ, GATHER>;
     if (!encode_rows(&prm.tmap_q, q, rows, D, MQ) || !encode_rows(&prm.tmap_k, k, rows, D, 1) ||
         !encode_rows(&prm.tmap_k16, k, rows, D, 16) || !encode_rows(&prm.tmap_v16, v, rows, D, 16))
         return FGATTN_ERR_CUDA;
@@ -66,14 +66,14 @@ fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const void* k, c
     const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;
     static bool configured = false;  // per process; the attribute is per function
     if (!configured) {
-        if (cudaFuncSetAttribute(fgattn::fgattn_fwd_kernel<D, MQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(fgattn::fgattn_fwd_kernel<D, MQ, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem) != cudaSuccess)
             return FGATTN_ERR_CUDA;
         // The warp roles re-divide the block's registers with setmaxnreg, which only
         // completes if the launch allocates exactly the per-thread count the split
         // was sized for: refuse to launch otherwise (it would wait forever).
         cudaFuncAttributes attr;
-        if (cudaFuncGetAttributes(&attr, fgattn::fgattn_fwd_kernel<D, MQ>) != cudaSuccess) return FGATTN_ERR_CUDA;
+        if (cudaFuncGetAttributes(&attr, fgattn::fgattn_fwd_kernel<D, MQ, GATHER>) != cudaSuccess) return FGATTN_ERR_CUDA;
         const bool split = C::SOFT_REGS != C::LAUNCH_REGS || C::AUX_REGS != C::LAUNCH_REGS;
         if (split && attr.numRegs != (int)C::LAUNCH_REGS) return FGATTN_ERR_UNSUPPORTED;
         configured = true;
@@ -81,8 +81,19 @@ fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const void* k, c
     const int sms = current_sms();
     if (sms <= 0) return FGATTN_ERR_CUDA;
     const int64_t grid = prm.items < sms ? prm.items : sms;
-    fgattn::fgattn_fwd_kernel<D, MQ><<<(unsigned)grid, C::THREADS, smem, stream>>>(prm);
+    fgattn::fgattn_fwd_kernel<D, MQ, GATHER><<<(unsigned)grid, C::THREADS, smem, stream>>>(prm);
     return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
+}
+
+template <int D, bool GATHER>
+fgattn_status dispatch_m(fgattn::FwdParams& prm, const void* q, const void* k, const void* v, int64_t rows, int64_t M,
+                         cudaStream_t s) {
+    switch (M) {
+        case 16: return launch_fwd<D, 16, GATHER>(prm, q, k, v, rows, s);
+        case 32: return launch_fwd<D, 32, GATHER>(prm, q, k, v, rows, s);
+        case 64: return launch_fwd<D, 64, GATHER>(prm, q, k, v, rows, s);
+        default: return launch_fwd<D, 128, GATHER>(prm, q, k, v, rows, s);
+    }
 }
 
 }  // namespace
@@ -143,24 +154,14 @@ fgattn_status fgattn_forward(const void* q, const void* k, const void* v, const 
     prm.QB = (L + M - 1) / M;
     prm.items = B * H * prm.QB;
     prm.scale_log2 = scale * 1.4426950408889634f;
-    (void)N;  // the key lists already encode the tile width
-
+    // Lists of whole 16-key runs (N a multiple of 16) load as TMA tiles: tile layout.
+    // Anything else is gathered row by row: gather layout (more K producer warps).
+    const bool gather = kept_idx != nullptr && N % 16 != 0;
     cudaStream_t s = (cudaStream_t)stream;
     const int64_t rows = B * H * L;
-    if (d == 128) {
-        switch (M) {
-            case 16: return launch_fwd<128, 16>(prm, q, k, v, rows, s);
-            case 32: return launch_fwd<128, 32>(prm, q, k, v, rows, s);
-            case 64: return launch_fwd<128, 64>(prm, q, k, v, rows, s);
-            default: return launch_fwd<128, 128>(prm, q, k, v, rows, s);
-        }
-    }
-    switch (M) {
-        case 16: return launch_fwd<64, 16>(prm, q, k, v, rows, s);
-        case 32: return launch_fwd<64, 32>(prm, q, k, v, rows, s);
-        case 64: return launch_fwd<64, 64>(prm, q, k, v, rows, s);
-        default: return launch_fwd<64, 128>(prm, q, k, v, rows, s);
-    }
+    if (d == 128)
+        return gather ? dispatch_m<128, true>(prm, q, k, v, rows, M, s) : dispatch_m<128, false>(prm, q, k, v, rows, M, s);
+    return gather ? dispatch_m<64, true>(prm, q, k, v, rows, M, s) : dispatch_m<64, false>(prm, q, k, v, rows, M, s);
 }
 
 fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* bits) {
