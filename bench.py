@@ -404,7 +404,8 @@ def main():
     traffic, _ = ncu_traffic(profile_key(w, args), _build.kernel_hash("fwd"))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                "peak_kind": f"{peak_kind} bf16 burst", "kernel": f"fgattn_fwd_kernel<{d},{M}>",
+                "peak_kind": f"{peak_kind} bf16 burst",
+                "kernel": f"fgattn_fwd_kernel<{d},{M},{'false' if (args.dense or N % 16 == 0) else 'true'}>",
                 "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "flops_per_launch": flops_per_step}
 
