@@ -22,7 +22,7 @@ import torch
 
 from . import _build
 
-__all__ = ["kept_capacity", "compact_mask", "forward", "device_error", "status_string", "num_sms",
+__all__ = ["kept_capacity", "compact_mask", "forward", "masked_forward_noalloc", "device_error", "status_string", "num_sms",
            "FgattnError", "LIB_PATH", "DEVERR_BAD_INDEX", "DEVERR_BAD_COUNT", "DEVERR_TIMEOUT"]
 
 LIB_PATH = _build.LIB
@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
     lib.fgattn_compact_mask.restype = i32
     lib.fgattn_forward.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float, p, p, p]
     lib.fgattn_forward.restype = i32
+    lib.fgattn_masked_forward_noalloc.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64, ctypes.c_float, p, p, p]
+    lib.fgattn_masked_forward_noalloc.restype = i32
     lib.fgattn_device_error.argtypes = [p, i32, ctypes.POINTER(ctypes.c_uint32)]
     lib.fgattn_device_error.restype = i32
     lib.fgattn_num_sms.argtypes = []
@@ -142,6 +144,30 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kept_idx: Optiona
         cap = L
     st = _lib.fgattn_forward(qp, kp, vp, ip, cp, cap, B, H, L, d, M, N, scale, op, lp, _stream_ptr(stream))
     _check(st, "fgattn_forward")
+    return out, lse
+
+
+def masked_forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: torch.Tensor, M: int, N: int,
+                           scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                           lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Mask -> (out, lse) with the kept lists in the library's fixed scratch array.
+
+    For callers that cannot allocate device memory: pass preallocated out and
+    lse and nothing is allocated (the library's array is at most
+    FGATTN_NOALLOC_SCRATCH_BYTES; larger problems raise FgattnError CAPACITY).
+    Calls that can overlap on the GPU share that array and race."""
+    B, H, L, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    bf = (torch.bfloat16,)
+    st = _lib.fgattn_masked_forward_noalloc(_dev(q, "q", bf), _dev(k, "k", bf), _dev(v, "v", bf),
+                                            _dev(mask, "mask", (torch.int32, torch.uint32)), B, H, L, d, M, N,
+                                            scale, _dev(out, "out", bf), _dev(lse, "lse", (torch.float32,)),
+                                            _stream_ptr(stream))
+    _check(st, "fgattn_masked_forward_noalloc")
     return out, lse
 
 

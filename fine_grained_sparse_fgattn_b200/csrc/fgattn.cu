@@ -191,3 +191,77 @@ const char* fgattn_status_string(fgattn_status status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Mask-driven forward for callers that cannot allocate device memory.
+//
+// Some callers are handed their input and output buffers and nothing else: a
+// plug-in running inside another runtime that owns the device's memory, or a
+// process whose memory is all reserved by a caching allocator, or code that
+// must not allocate once set-up is over.  For them the kept lists that
+// fgattn_compact_mask writes and fgattn_forward reads live in one fixed
+// array that the library itself holds on every device that loads it.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace {
+
+// Kept-list scratch: the counts first (rows rounded up to 64 entries, so the
+// lists that follow start 256-byte aligned), then rows x cap kept indices.
+// Nothing in it has to start at zero: the compaction writes every count and
+// the first `count` entries of every list, and the forward reads no more.
+static __device__ __align__(256) int32_t g_noalloc_scratch[FGATTN_NOALLOC_SCRATCH_BYTES / sizeof(int32_t)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+int32_t* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// g_noalloc_scratch names a host-side stand-in, never the device copy.
+fgattn_status noalloc_scratch(int32_t** ptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FGATTN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FGATTN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FGATTN_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return FGATTN_OK;
+}
+
+}  // namespace
+
+extern "C" fgattn_status fgattn_masked_forward_noalloc(const void* q, const void* k, const void* v,
+                                                       const uint32_t* mask, int64_t B, int64_t H, int64_t L,
+                                                       int64_t d, int64_t M, int64_t N, float scale, void* out,
+                                                       float* lse, fgattn_stream_t stream) {
+    // Every check of both steps comes first, so an error status means nothing was enqueued.
+    if (!q || !k || !v || !out || !mask) return FGATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || L < 1 || M < 1 || N < 1 || d < 1) return FGATTN_ERR_INVALID_ARG;
+    if (L > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return FGATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FGATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(mask) & 3u) return FGATTN_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FGATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;
+    const int64_t cap = fgattn_kept_capacity(L);
+    const int64_t rows = B * H * ((L + M - 1) / M);
+    const int64_t cnt_entries = (rows + 63) / 64 * 64;
+    const int64_t limit = (int64_t)(FGATTN_NOALLOC_SCRATCH_BYTES / sizeof(int32_t));
+    if (rows > limit || cap > limit || cnt_entries + rows * cap > limit) return FGATTN_ERR_CAPACITY;
+
+    int32_t* scratch = nullptr;
+    const fgattn_status st = noalloc_scratch(&scratch);
+    if (st != FGATTN_OK) return st;
+    int32_t* kept_cnt = scratch;
+    int32_t* kept_idx = scratch + cnt_entries;
+    const fgattn_status sc = fgattn_compact_mask(mask, B, H, L, M, N, kept_idx, kept_cnt, cap, stream);
+    if (sc != FGATTN_OK) return sc;
+    return fgattn_forward(q, k, v, kept_idx, kept_cnt, cap, B, H, L, d, M, N, scale, out, lse, stream);
+}

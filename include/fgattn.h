@@ -117,6 +117,44 @@ fgattn_status fgattn_forward(const void* q, const void* k, const void* v, const 
  */
 fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* bits);
 
+/*
+ * Size of the kept-list scratch array that fgattn_masked_forward_noalloc
+ * uses: 64 MiB, held on every device that loads the library, until exit.
+ */
+#define FGATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * Mask to attention output without any device allocation: fgattn_compact_mask
+ * followed by fgattn_forward, with the kept lists in a fixed scratch array
+ * inside the library instead of caller memory.  The paper has no counterpart;
+ * this entry point exists for callers that cannot allocate device memory
+ * themselves (a plug-in handed only its input and output buffers by the
+ * runtime that hosts it, a process whose device memory is all reserved by a
+ * caching allocator, code that must not allocate once set-up is over).
+ *   q, k, v   in   device bf16 [B][H][L][d]
+ *   mask      in   device uint32 [B][H][QB][W]  (layout and diagonal rule as above)
+ *   out       out  device bf16 [B][H][L][d]
+ *   lse       out  device fp32 [B][H][L], may be NULL
+ * Results equal fgattn_compact_mask + fgattn_forward on the same arguments.
+ * Limit: the kept lists take 4 * (ceil(R / 64) * 64 + R * cap) bytes, with
+ * R = B * H * QB rows and cap = fgattn_kept_capacity(L); a call that needs
+ * more than FGATTN_NOALLOC_SCRATCH_BYTES returns CAPACITY and enqueues nothing
+ * (for example B = 1, H = 8, L = 8192, M = 64 needs 32 MiB and fits).
+ * No cudaMalloc, cudaFree or other allocating call is made.
+ * Set-up: the first call on a device looks up that device's address of the
+ * array (with the device current); make that first call before any stream
+ * capture begins.
+ * Sharing: every call on a device uses the same array, and it keeps the last
+ * call's lists.  Calls in one stream are ordered and safe; calls that can run
+ * at the same time on the GPU (different streams, no ordering between them)
+ * race on the array and give wrong results.
+ * Errors: INVALID_ARG, UNSUPPORTED, CAPACITY, CUDA; device-side problems as
+ * for fgattn_forward.
+ */
+fgattn_status fgattn_masked_forward_noalloc(const void* q, const void* k, const void* v, const uint32_t* mask,
+                                            int64_t B, int64_t H, int64_t L, int64_t d, int64_t M, int64_t N,
+                                            float scale, void* out, float* lse, fgattn_stream_t stream);
+
 /* Number of streaming multiprocessors the forward kernel's persistent grid uses
  * on the current device (0 on failure). */
 int fgattn_num_sms(void);

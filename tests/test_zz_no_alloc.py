@@ -1,0 +1,75 @@
+"""The allocation-free entry point, fgattn_masked_forward_noalloc, against the
+usual two-call path (fgattn_compact_mask into caller buffers, then
+fgattn_forward).
+
+The entry point exists for callers that are given their input and output
+buffers and cannot allocate device memory themselves (a plug-in inside a
+runtime that owns the device's memory, a process whose memory is all held by a
+caching allocator, code that must not allocate after set-up).  It keeps the
+kept lists in one fixed array inside the library instead.
+
+Two calls in a row: the first (per-key layer, 8 heads, 32 MiB of lists) fills
+most of the array; the second is a different shape with short lists, so stale
+entries of the first call lie past every new count and must not be read.
+This file is collected last so that a stop-at-first-failure run has already
+run every other test.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fine_grained_sparse_fgattn_b200 as F
+import workloads as W
+from gpu_common import LSE_MAX_ABS, OUT_MAX_ABS, OUT_REL_RMS
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(q, k, v, mask, M, N, scale, out, lse):
+    B, H, L, d = q.shape
+    return F._lib.fgattn_masked_forward_noalloc(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), mask.data_ptr(), B, H, L, d, M, N, scale,
+        out.data_ptr(), lse.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+
+def _case(q, k, v, mask_np, M, N):
+    dev = torch.device("cuda", 0)
+    B, H, L, d = q.shape
+    scale = 1.0 / np.sqrt(d)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    md = torch.from_numpy(mask_np.view(np.int32)).to(dev)
+    # Existing entry points, caller-allocated lists.
+    idx, cnt = F.compact_mask(md, B, H, L, M, N)
+    o_ref, l_ref = F.forward(qd, kd, vd, idx, cnt, M, N, scale)
+    # The allocation-free entry point, outputs pre-filled with NaN.
+    out = torch.full_like(qd, float("nan"))
+    lse = torch.full((B, H, L), float("nan"), dtype=torch.float32, device=dev)
+    assert _noalloc(qd, kd, vd, md, M, N, scale, out, lse) == F.OK
+    assert F.device_error() == 0
+    return out.float().cpu().numpy(), lse.cpu().numpy(), o_ref.float().cpu().numpy(), l_ref.cpu().numpy()
+
+
+def _check(o, l, o_ref, l_ref):
+    assert np.isfinite(o).all() and np.isfinite(l).all()
+    assert np.abs(o - o_ref).max() <= OUT_MAX_ABS
+    assert np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref) <= OUT_REL_RMS
+    assert np.abs(l - l_ref).max() <= LSE_MAX_ABS
+
+
+def test_noalloc_matches_two_call_path_twice_in_a_row():
+    w = W.get("perkey")  # B1 H8 L8192 d128, M64 N1: 32 MiB of kept lists
+    q, k, v = W.make_qkv(w, 0)
+    _check(*_case(q, k, v, W.make_mask(w, 0), w.M, w.N))
+
+    B, H, L, d, M, N = 1, 3, 700, 128, 64, 16
+    QB, G = -(-L // M), -(-L // N)
+    q, k, v = W.random_qkv(B, H, L, d, seed=5)
+    mask = W.pack_tiles(W.random_tiles(B, H, QB, G, 0.1, seed=6))
+    _check(*_case(q, k, v, mask, M, N))
+
+
+def test_noalloc_refuses_sizes_beyond_its_array():
+    P = 1 << 20  # never dereferenced: the size check refuses the call first
+    # Wan-480p-like layer: 40 heads x 512 blocks x 32768 entries, far above 64 MiB.
+    st = F._lib.fgattn_masked_forward_noalloc(P, P, P, P, 1, 40, 32760, 128, 64, 16, 0.088, P, P, None)
+    assert st == F.ERR_CAPACITY
