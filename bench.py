@@ -242,12 +242,14 @@ def cfg_dict(w, args, flush):
     return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "grid": list(w.grid), "d": w.d, "M": w.M, "N": w.N,
             "sparsity_target": w.sparsity, "mask": w.mask, "qkv": w.qkv, "seed": args.seed,
             "l2": l2, "parallelism": f"heads x{args.gpus} (weak)",
-            "path": "dense (no kept lists)" if getattr(args, "dense", False) else "tile-sparse (compaction + forward)"}
+            "path": "dense (no kept lists)" if getattr(args, "dense", False) else "tile-sparse (compaction + forward)",
+            "layout": "[B][L][H][d]" if getattr(args, "layout", "bhld") == "blhd" else "[B][H][L][d]"}
 
 
 def profile_key(w, args):
     """Name of the committed ncu summary for this exact workload (None when overridden)."""
-    if args.N is not None or args.sparsity is not None or args.heads is not None or args.dense:
+    if args.N is not None or args.sparsity is not None or args.heads is not None or args.dense or \
+            args.layout != "bhld":
         return None
     return w.name
 
@@ -266,6 +268,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layout", default="bhld", choices=["bhld", "blhd"],
+                    help="memory layout of q, k, v, out: [B][H][L][d] (contiguous entry point) or "
+                         "[B][L][H][d] (strided entry point)")
     ap.add_argument("--dense", action="store_true",
                     help="dense run of the same kernel (no kept lists: every key of every block)")
     args = ap.parse_args()
@@ -290,8 +295,11 @@ def main():
 
     # ---- inputs: seeded on the host, then resident in HBM before timing
     q_h, k_h, v_h = W.make_qkv(w, args.seed, heads=heads)
+    if args.layout == "blhd":  # [B][L][H][d] storage, used through [B][H][L][d] views
+        q_h, k_h, v_h = (t.transpose(1, 2).contiguous().transpose(1, 2) for t in (q_h, k_h, v_h))
     mask_h = W.make_mask(w, args.seed, heads=heads)
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    q, k, v = (t.transpose(1, 2).to(dev).transpose(1, 2) if args.layout == "blhd" else t.to(dev)
+               for t in (q_h, k_h, v_h))
     mask = torch.from_numpy(mask_h.view(np.int32)).to(dev)
     cap = F.kept_capacity(L)
     kept_idx = torch.empty((B, H, QB, cap), dtype=torch.int32, device=dev)
@@ -368,9 +376,13 @@ def main():
     value = job_throughput(world, flops_per_step, ms_per_step)
 
     # ---- end to end through the public API: pinned host inputs -> device -> host results
-    qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    if args.layout == "blhd":
+        qp, kp, vp = (t.transpose(1, 2).pin_memory().transpose(1, 2) for t in (q_h, k_h, v_h))
+    else:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
     mp = torch.from_numpy(mask_h.view(np.int32)).pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    out_h = torch.empty_like(out, device="cpu").pin_memory() if args.layout == "bhld" else \
+        torch.empty((B, L, H, d), dtype=out.dtype).pin_memory().transpose(1, 2)
     lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (qp, kp, vp, mp))
     d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()

@@ -45,6 +45,9 @@ def _load() -> ctypes.CDLL:
     lib.fgattn_compact_mask.restype = i32
     lib.fgattn_forward.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float, p, p, p]
     lib.fgattn_forward.restype = i32
+    lib.fgattn_forward_strided.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64,
+                                           ctypes.c_float, p, p, p, p]
+    lib.fgattn_forward_strided.restype = i32
     lib.fgattn_masked_forward_noalloc.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64, ctypes.c_float, p, p, p]
     lib.fgattn_masked_forward_noalloc.restype = i32
     lib.fgattn_device_error.argtypes = [p, i32, ctypes.POINTER(ctypes.c_uint32)]
@@ -89,6 +92,18 @@ def _dev(t: torch.Tensor, name: str, dtypes) -> int:
     return t.data_ptr()
 
 
+def _dev_rows(t: torch.Tensor, name: str):
+    """A [B, H, L, d] bf16 view whose last dimension is contiguous: (pointer, host int64[3] strides)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected torch.bfloat16")
+    if t.dim() != 4 or (t.shape[-1] > 1 and t.stride(-1) != 1):
+        raise ValueError(f"{name} must be a [B, H, L, d] view with a contiguous last dimension")
+    st = (ctypes.c_int64 * 3)(*t.stride()[:3])
+    return t.data_ptr(), st
+
+
 def kept_capacity(L: int) -> int:
     """Per-row stride of kept_idx: L rounded up to 16."""
     return int(_lib.fgattn_kept_capacity(int(L)))
@@ -122,6 +137,9 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kept_idx: Optiona
             stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Tile-sparse attention forward.  q, k, v: bf16 [B,H,L,d].  kept_idx None = dense run.
 
+    q, k, v and out may be any [B,H,L,d] views with a contiguous last dimension
+    (e.g. x.transpose(1, 2) of a [B,L,H,d] tensor, or slices of a packed
+    [B,L,3,H,d] projection); out defaults to the layout of q.
     Returns (out bf16 [B,H,L,d], lse fp32 [B,H,L] natural-log, or None)."""
     if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must share one [B, H, L, d] shape")
@@ -129,12 +147,19 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kept_idx: Optiona
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     if out is None:
         out = torch.empty_like(q)
+    if out.shape != q.shape:
+        raise ValueError("out must have the shape of q")
     if lse is None and want_lse:
         lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
-    bf = (torch.bfloat16,)
-    qp, kp, vp = _dev(q, "q", bf), _dev(k, "k", bf), _dev(v, "v", bf)
-    op = _dev(out, "out", bf)
     lp = _dev(lse, "lse", (torch.float32,)) if lse is not None else None
+    strided = not all(t.is_contiguous() for t in (q, k, v, out))
+    if strided:
+        (qp, qs), (kp, ks), (vp, vs), (op, os_) = (_dev_rows(t, n) for t, n in
+                                                   ((q, "q"), (k, "k"), (v, "v"), (out, "out")))
+    else:
+        bf = (torch.bfloat16,)
+        qp, kp, vp = _dev(q, "q", bf), _dev(k, "k", bf), _dev(v, "v", bf)
+        op = _dev(out, "out", bf)
     if kept_idx is not None:
         ip = _dev(kept_idx, "kept_idx", (torch.int32,))
         cp = _dev(kept_cnt, "kept_cnt", (torch.int32,))
@@ -142,8 +167,13 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kept_idx: Optiona
     else:
         ip = cp = None
         cap = L
-    st = _lib.fgattn_forward(qp, kp, vp, ip, cp, cap, B, H, L, d, M, N, scale, op, lp, _stream_ptr(stream))
-    _check(st, "fgattn_forward")
+    if strided:
+        st = _lib.fgattn_forward_strided(qp, qs, kp, ks, vp, vs, ip, cp, cap, B, H, L, d, M, N, scale, op, os_, lp,
+                                         _stream_ptr(stream))
+        _check(st, "fgattn_forward_strided")
+    else:
+        st = _lib.fgattn_forward(qp, kp, vp, ip, cp, cap, B, H, L, d, M, N, scale, op, lp, _stream_ptr(stream))
+        _check(st, "fgattn_forward")
     return out, lse
 
 

@@ -62,12 +62,28 @@ constexpr uint32_t kErrBadCount = 0x2u;
 constexpr uint32_t kErrTimeout = 0x4u;
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 
+// Layouts (template parameter STRIDED).  Contiguous: q, k, v, out are
+// [B][H][L][D]; the tile maps (q, k16, v16) and the gather map (k) are 2-D over
+// the B*H*L rows.  Strided: q, k, v, out are [B][H][L][D] views with D
+// contiguous and element strides (sb, sh, sl) in any order in memory
+// ([B][L][H][D], a packed [B][L][3][H][D] projection ...); the tile maps are
+// 4-D {D, L, H, B} with coordinates (x, l, h, b), and the gather map over k and
+// the cp.async row copies of v count in rows of D elements (every stride is a
+// whole number of rows).  The contiguous kernel is kept separate because its
+// copy loops are sensitive to their code size: the general addressing measured
+// 4-8 % slower on the sparse forward.
 struct alignas(64) FwdParams {
-    CUtensorMap tmap_q;  // [B*H*L rows][D], box {64, MQ}, 128B swizzle
-    CUtensorMap tmap_k;    // [B*H*L rows][D], box {64, 1},  128B swizzle (row gathers)
-    CUtensorMap tmap_k16;  // [B*H*L rows][D], box {64, 16}, 128B swizzle (16 consecutive rows)
+    CUtensorMap tmap_q;    // q tiles: box {64, MQ} (contiguous) or {64, MQ, 1, 1} (strided), 128B swizzle
+    CUtensorMap tmap_k;    // k rows of D elements, box {64, 1} (row gathers)
+    CUtensorMap tmap_k16;  // k tiles: box {64, 16} or {64, 16, 1, 1} (16 consecutive keys)
     CUtensorMap tmap_v16;  // same for V
     const __nv_bfloat16* v_base;  // V rows, gathered with cp.async where not consecutive
+    // strided layout only
+    int64_t k_ub, k_uh;  // k batch / head strides in rows of D elements
+    int64_t v_ub, v_uh;  // v batch / head strides in rows of D elements
+    int32_t k_ul, v_ul;  // k / v token strides in rows of D elements
+    int64_t o_sb, o_sh, o_sl;  // out element strides
+    int64_t H;
     const int32_t* kept_idx;  // nullptr: dense (every key kept)
     const int32_t* kept_cnt;
     __nv_bfloat16* out;
@@ -222,9 +238,10 @@ __device__ __forceinline__ int4 fetch_idx(const int32_t* lst, int64_t cnt, int64
                      j0 + 2 < cnt ? __ldg(lst + j0 + 2) : 0, j0 + 3 < cnt ? __ldg(lst + j0 + 3) : 0);
 }
 
-// Global row coordinates of four fetched entries.  Entries outside [0, L) are
-// reported and replaced by key 0 of the head (as are entries past the list,
-// whose scores the softmax masks).
+// Gather-map row coordinates of four fetched entries: row0 + key * stride.
+// Entries outside [0, L) are reported and replaced by key 0 of the head (as are
+// entries past the list, whose scores the softmax masks).
+template <bool STRIDED>
 __device__ __forceinline__ void rows_of(const FwdParams& p, int4 raw, int64_t row0, bool report, int32_t (&rows)[4]) {
     const int32_t idx[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
@@ -234,11 +251,14 @@ __device__ __forceinline__ void rows_of(const FwdParams& p, int4 raw, int64_t ro
             if (report) atomicOr(&g_device_error, kErrBadIndex);
             x = 0;
         }
-        rows[i] = (int32_t)(row0 + x);
+        if constexpr (STRIDED)
+            rows[i] = (int32_t)row0 + x * p.k_ul;
+        else
+            rows[i] = (int32_t)(row0 + x);
     }
 }
 
-template <int D, int MQ, bool GATHER>
+template <int D, int MQ, bool GATHER, bool STRIDED>
 __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
     fgattn_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = FwdCfg<D, MQ, GATHER>;
@@ -312,6 +332,13 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
         for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
             const int64_t bh = item / p.QB;
             const int64_t qb = item - bh * p.QB;
+            int32_t bi = 0, hi = 0;
+            int64_t krow0 = bh * L;  // first gather-map row of this head's keys
+            if constexpr (STRIDED) {
+                bi = (int32_t)(bh / p.H);
+                hi = (int32_t)(bh - (int64_t)bi * p.H);
+                krow0 = bi * p.k_ub + hi * p.k_uh;
+            }
             const int64_t cnt = item_count(p, item, kw == 0 && lane == 0);
             const int64_t nch = (cnt + 127) / 128;
             const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
@@ -325,8 +352,12 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                     ptx::mbar_arrive_expect_tx(BAR(C::B_QFULL), (uint32_t)C::Q_TILE);
 #pragma unroll
                     for (int pn = 0; pn < D / 64; ++pn)
-                        ptx::tma_load_2d(QTILE + (uint32_t)pn * (MQ * 128), &p.tmap_q, pn * 64,
-                                         (int32_t)(bh * L + qb * MQ), BAR(C::B_QFULL));
+                        if constexpr (STRIDED)
+                            ptx::tma_load_4d(QTILE + (uint32_t)pn * (MQ * 128), &p.tmap_q, pn * 64,
+                                             (int32_t)(qb * MQ), hi, bi, BAR(C::B_QFULL));
+                        else
+                            ptx::tma_load_2d(QTILE + (uint32_t)pn * (MQ * 128), &p.tmap_q, pn * 64,
+                                             (int32_t)(bh * L + qb * MQ), BAR(C::B_QFULL));
                 }
                 ++q_issued;
                 __syncwarp();
@@ -365,12 +396,16 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                         if ((lane & 3) == 0) {
 #pragma unroll
                             for (int pn = 0; pn < D / 64; ++pn)
-                                ptx::tma_load_2d(dst + (uint32_t)pn * (128 * 128), &p.tmap_k16, pn * 64,
-                                                 (int32_t)(bh * L + first), BAR(C::B_KFULL + st));
+                                if constexpr (STRIDED)
+                                    ptx::tma_load_4d(dst + (uint32_t)pn * (128 * 128), &p.tmap_k16, pn * 64, first,
+                                                     hi, bi, BAR(C::B_KFULL + st));
+                                else
+                                    ptx::tma_load_2d(dst + (uint32_t)pn * (128 * 128), &p.tmap_k16, pn * 64,
+                                                     (int32_t)(bh * L + first), BAR(C::B_KFULL + st));
                         }
                     } else {
                         int32_t rows[4];
-                        rows_of(p, cur, bh * L, true, rows);
+                        rows_of<STRIDED>(p, cur, krow0, true, rows);
 #pragma unroll
                         for (int pn = 0; pn < D / 64; ++pn)
                             ptx::tma_gather4(dst + (uint32_t)pn * (128 * 128), &p.tmap_k, pn * 64, rows[0], rows[1],
@@ -400,6 +435,12 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
             const int64_t nch = (cnt + 127) / 128;
             const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
             const __nv_bfloat16* vb = p.v_base + (size_t)bh * L * D;
+            int32_t bi = 0, hi = 0, vrow0 = 0;
+            if constexpr (STRIDED) {
+                bi = (int32_t)(bh / p.H);
+                hi = (int32_t)(bh - (int64_t)bi * p.H);
+                vrow0 = (int32_t)(bi * p.v_ub + hi * p.v_uh);  // first row (of D elements) of this head
+            }
             auto fetch1 = [&](int64_t c) -> int32_t {
                 const int64_t j = c * 128 + vw * 32 + lane;
                 if (j >= cnt) return -1;  // past the list
@@ -437,9 +478,14 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                         if (lane == 0) {
                             ptx::mbar_expect_tx(BAR(C::B_VFULL + st), (uint32_t)(16 * D * 2));
 #pragma unroll
-                            for (int pn = 0; pn < D / 64; ++pn)
-                                ptx::tma_load_2d(vdst + (uint32_t)pn * (128 * 128) + (uint32_t)r0 * 128u, &p.tmap_v16,
-                                                 pn * 64, (int32_t)(bh * L + fs), BAR(C::B_VFULL + st));
+                            for (int pn = 0; pn < D / 64; ++pn) {
+                                if constexpr (STRIDED)
+                                    ptx::tma_load_4d(vdst + (uint32_t)pn * (128 * 128) + (uint32_t)r0 * 128u,
+                                                     &p.tmap_v16, pn * 64, fs, hi, bi, BAR(C::B_VFULL + st));
+                                else
+                                    ptx::tma_load_2d(vdst + (uint32_t)pn * (128 * 128) + (uint32_t)r0 * 128u,
+                                                     &p.tmap_v16, pn * 64, (int32_t)(bh * L + fs), BAR(C::B_VFULL + st));
+                            }
                         }
                     } else {
 #pragma unroll
@@ -448,8 +494,12 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                             const int pc = lane % PPR;
                             const int32_t ridx = __shfl_sync(0xffffffffu, idx, rl);
                             const int r = vw * 32 + rl;
-                            ptx::cp_async_16(vdst + (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128),
-                                             vb + (size_t)ridx * D + pc * 8, 16u);
+                            const __nv_bfloat16* src;
+                            if constexpr (STRIDED)
+                                src = p.v_base + (size_t)(uint32_t)(vrow0 + ridx * p.v_ul) * D + pc * 8;
+                            else
+                                src = vb + (size_t)ridx * D + pc * 8;
+                            ptx::cp_async_16(vdst + (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128), src, 16u);
                         }
                     }
                 }
@@ -737,6 +787,12 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
             }
             ptx::named_sync(nbar, 128);
             __nv_bfloat16* outb = p.out + (size_t)bh * L * D;
+            int64_t ostride = D;  // elements between consecutive query rows of out
+            if constexpr (STRIDED) {
+                const int64_t bi = bh / p.H;
+                outb = p.out + bi * p.o_sb + (bh - bi * p.H) * p.o_sh;
+                ostride = p.o_sl;
+            }
             constexpr int SR = C::SROWS;
 #pragma unroll 1
             for (int q0 = 0; q0 < CW; q0 += SR) {
@@ -757,7 +813,7 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                     const int64_t row = qb * MQ + col0 + q0 + r;
                     if (row < L) {
                         const uint4 val = *reinterpret_cast<const uint4*>(stage + r * D + pc * 8);
-                        *reinterpret_cast<uint4*>(outb + row * D + pc * 8) = val;
+                        *reinterpret_cast<uint4*>(outb + row * ostride + pc * 8) = val;
                     }
                 }
                 ptx::named_sync(nbar, 128);

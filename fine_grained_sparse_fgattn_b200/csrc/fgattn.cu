@@ -32,18 +32,39 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Row-major bf16 matrix [rows][d] viewed in boxes of 64 columns x box_rows rows, 128B swizzle.
-bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t d, uint32_t box_rows) {
+// bf16 rows of d elements, `row_stride` elements apart, viewed in boxes of 64 columns x
+// box_rows rows, 128B swizzle.
+bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t d, int64_t row_stride, uint32_t box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
     const cuuint32_t box[2] = {64u, box_rows};
     const cuuint32_t estr[2] = {1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// [B][H][L][d] view with element strides st = {sb, sh, sl} (d contiguous) as a 4-D
+// map {d, L, H, B} in boxes of 64 columns x box_rows consecutive L positions, 128B swizzle.
+bool encode_4d(CUtensorMap* m, const void* base, int64_t B, int64_t H, int64_t L, int64_t d, const int64_t* st,
+               uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
+    const cuuint32_t box[4] = {64u, box_rows, 1u, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Strides of one tensor, in elements: {batch, head, token}.
+struct Strides {
+    int64_t s[3];
+};
 
 int current_sms() {
     int dev = 0;
@@ -53,27 +74,35 @@ int current_sms() {
     return sms;
 }
 
-template <int D, int MQ, bool GATHER>
-fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const void* k, const void* v, int64_t rows,
+template <int D, int MQ, bool GATHER, bool STRIDED>
+fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
+                         const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows,
                          cudaStream_t stream) {
     using C = fgattn::FwdCfg<D, MQ, GATHER>;
-    if (!encode_rows(&prm.tmap_q, q, rows, D, MQ) || !encode_rows(&prm.tmap_k, k, rows, D, 1) ||
-        !encode_rows(&prm.tmap_k16, k, rows, D, 16) || !encode_rows(&prm.tmap_v16, v, rows, D, 16))
-        return FGATTN_ERR_CUDA;
-    prm.v_base = static_cast<const __nv_bfloat16*>(v);
+    const int64_t L = prm.L;
+    if (STRIDED) {
+        if (!encode_4d(&prm.tmap_q, q, B, H, L, D, qs.s, MQ) || !encode_rows(&prm.tmap_k, k, k_rows, D, D, 1) ||
+            !encode_4d(&prm.tmap_k16, k, B, H, L, D, ks.s, 16) || !encode_4d(&prm.tmap_v16, v, B, H, L, D, vs.s, 16))
+            return FGATTN_ERR_CUDA;
+    } else {
+        const int64_t rows = B * H * L;
+        if (!encode_rows(&prm.tmap_q, q, rows, D, D, MQ) || !encode_rows(&prm.tmap_k, k, rows, D, D, 1) ||
+            !encode_rows(&prm.tmap_k16, k, rows, D, D, 16) || !encode_rows(&prm.tmap_v16, v, rows, D, D, 16))
+            return FGATTN_ERR_CUDA;
+    }
+    auto kernel = fgattn::fgattn_fwd_kernel<D, MQ, GATHER, STRIDED>;
     // Request enough shared memory that exactly one block is resident per SM:
     // the grid is persistent (one block per SM, static round-robin over work).
     const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;
     static bool configured = false;  // per process; the attribute is per function
     if (!configured) {
-        if (cudaFuncSetAttribute(fgattn::fgattn_fwd_kernel<D, MQ, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem) != cudaSuccess)
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return FGATTN_ERR_CUDA;
         // The warp roles re-divide the block's registers with setmaxnreg, which only
         // completes if the launch allocates exactly the per-thread count the split
         // was sized for: refuse to launch otherwise (it would wait forever).
         cudaFuncAttributes attr;
-        if (cudaFuncGetAttributes(&attr, fgattn::fgattn_fwd_kernel<D, MQ, GATHER>) != cudaSuccess) return FGATTN_ERR_CUDA;
+        if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FGATTN_ERR_CUDA;
         const bool split = C::SOFT_REGS != C::LAUNCH_REGS || C::AUX_REGS != C::LAUNCH_REGS;
         if (split && attr.numRegs != (int)C::LAUNCH_REGS) return FGATTN_ERR_UNSUPPORTED;
         configured = true;
@@ -81,19 +110,91 @@ fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const void* k, c
     const int sms = current_sms();
     if (sms <= 0) return FGATTN_ERR_CUDA;
     const int64_t grid = prm.items < sms ? prm.items : sms;
-    fgattn::fgattn_fwd_kernel<D, MQ, GATHER><<<(unsigned)grid, C::THREADS, smem, stream>>>(prm);
+    kernel<<<(unsigned)grid, C::THREADS, smem, stream>>>(prm);
     return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
 }
 
-template <int D, bool GATHER>
-fgattn_status dispatch_m(fgattn::FwdParams& prm, const void* q, const void* k, const void* v, int64_t rows, int64_t M,
+template <int D, bool GATHER, bool STRIDED>
+fgattn_status dispatch_m(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
+                         const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows, int64_t M,
                          cudaStream_t s) {
     switch (M) {
-        case 16: return launch_fwd<D, 16, GATHER>(prm, q, k, v, rows, s);
-        case 32: return launch_fwd<D, 32, GATHER>(prm, q, k, v, rows, s);
-        case 64: return launch_fwd<D, 64, GATHER>(prm, q, k, v, rows, s);
-        default: return launch_fwd<D, 128, GATHER>(prm, q, k, v, rows, s);
+        case 16: return launch_fwd<D, 16, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
+        case 32: return launch_fwd<D, 32, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
+        case 64: return launch_fwd<D, 64, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
+        default: return launch_fwd<D, 128, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
     }
+}
+
+template <bool STRIDED>
+fgattn_status dispatch(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
+                       const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows, int64_t d, int64_t M,
+                       bool gather, cudaStream_t s) {
+    if (d == 128)
+        return gather ? dispatch_m<128, true, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
+                      : dispatch_m<128, false, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
+    return gather ? dispatch_m<64, true, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
+                  : dispatch_m<64, false, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
+}
+
+// Shared by fgattn_forward (contiguous [B][H][L][d]) and fgattn_forward_strided.
+fgattn_status forward_impl(const void* q, const Strides& qs, const void* k, const Strides& ks, const void* v,
+                           const Strides& vs, const int32_t* kept_idx, const int32_t* kept_cnt, int64_t cap, int64_t B,
+                           int64_t H, int64_t L, int64_t d, int64_t M, int64_t N, float scale, void* out,
+                           const Strides& os, float* lse, fgattn_stream_t stream) {
+    if (!q || !k || !v || !out) return FGATTN_ERR_INVALID_ARG;
+    if (kept_idx && !kept_cnt) return FGATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || L < 1 || M < 1 || N < 1 || d < 1) return FGATTN_ERR_INVALID_ARG;
+    if (L > INT32_MAX || B > INT32_MAX || H > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return FGATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FGATTN_ERR_INVALID_ARG;
+    if (kept_idx && !aligned16(kept_idx)) return FGATTN_ERR_INVALID_ARG;  // rows are read as int4
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FGATTN_ERR_INVALID_ARG;
+    if (kept_idx && (cap < L || (cap & 3))) return FGATTN_ERR_CAPACITY;
+    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
+    // Strides: at least one row (d) and 16-byte multiples (TMA, vector stores); k and v
+    // strides whole rows of d, so every key row is a row of the gather map over k.
+    const Strides* all[4] = {&qs, &ks, &vs, &os};
+    for (int t = 0; t < 4; ++t)
+        for (int i = 0; i < 3; ++i) {
+            const int64_t x = all[t]->s[i];
+            if (x < d || (x & 7) || x >= (int64_t(1) << 38)) return FGATTN_ERR_INVALID_ARG;
+            if (t >= 1 && t <= 2 && x % d) return FGATTN_ERR_INVALID_ARG;
+        }
+    const int64_t k_rows = ((B - 1) * ks.s[0] + (H - 1) * ks.s[1] + (L - 1) * ks.s[2]) / d + 1;
+    const int64_t v_rows = ((B - 1) * vs.s[0] + (H - 1) * vs.s[1] + (L - 1) * vs.s[2]) / d + 1;
+    // 32-bit TMA coordinates and row numbers in the kernels
+    if (k_rows > INT32_MAX || v_rows > INT32_MAX || B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;
+
+    fgattn::FwdParams prm;
+    prm.kept_idx = kept_idx;
+    prm.kept_cnt = kept_cnt;
+    prm.out = static_cast<__nv_bfloat16*>(out);
+    prm.lse = lse;
+    prm.cap = kept_idx ? cap : L;
+    prm.L = L;
+    prm.H = H;
+    prm.QB = (L + M - 1) / M;
+    prm.items = B * H * prm.QB;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.v_base = static_cast<const __nv_bfloat16*>(v);
+    prm.k_ub = ks.s[0] / d, prm.k_uh = ks.s[1] / d, prm.k_ul = (int32_t)(ks.s[2] / d);
+    prm.v_ub = vs.s[0] / d, prm.v_uh = vs.s[1] / d, prm.v_ul = (int32_t)(vs.s[2] / d);
+    prm.o_sb = os.s[0], prm.o_sh = os.s[1], prm.o_sl = os.s[2];
+    // Lists of whole 16-key runs (N a multiple of 16) load as TMA tiles: tile layout.
+    // Anything else is gathered row by row: gather layout (more K producer warps).
+    const bool gather = kept_idx != nullptr && N % 16 != 0;
+    // Contiguous [B][H][L][d] everywhere (strides of extent-1 dimensions aside): the
+    // contiguous kernel.
+    const Strides c = {{H * L * d, L * d, d}};
+    const int64_t extent[3] = {B, H, L};
+    bool contiguous = true;
+    for (const Strides* t : {&qs, &ks, &vs, &os})
+        for (int i = 0; i < 3; ++i) contiguous = contiguous && (extent[i] == 1 || t->s[i] == c.s[i]);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (contiguous) return dispatch<false>(prm, q, qs, k, ks, v, vs, B, H, k_rows, d, M, gather, s);
+    return dispatch<true>(prm, q, qs, k, ks, v, vs, B, H, k_rows, d, M, gather, s);
 }
 
 }  // namespace
@@ -131,37 +232,23 @@ fgattn_status fgattn_compact_mask(const uint32_t* mask, int64_t B, int64_t H, in
 fgattn_status fgattn_forward(const void* q, const void* k, const void* v, const int32_t* kept_idx,
                              const int32_t* kept_cnt, int64_t cap, int64_t B, int64_t H, int64_t L, int64_t d,
                              int64_t M, int64_t N, float scale, void* out, float* lse, fgattn_stream_t stream) {
-    if (!q || !k || !v || !out) return FGATTN_ERR_INVALID_ARG;
-    if (kept_idx && !kept_cnt) return FGATTN_ERR_INVALID_ARG;
-    if (B < 1 || H < 1 || L < 1 || M < 1 || N < 1 || d < 1) return FGATTN_ERR_INVALID_ARG;
-    if (L > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return FGATTN_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FGATTN_ERR_INVALID_ARG;
-    if (kept_idx && !aligned16(kept_idx)) return FGATTN_ERR_INVALID_ARG;  // rows are read as int4
-    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FGATTN_ERR_INVALID_ARG;
-    if (kept_idx && (cap < L || (cap & 3))) return FGATTN_ERR_CAPACITY;
-    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
-    if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (d < 1 || L < 1 || H < 1) return FGATTN_ERR_INVALID_ARG;
+    const Strides c = {{H * L * d, L * d, d}};  // contiguous [B][H][L][d]
+    return forward_impl(q, c, k, c, v, c, kept_idx, kept_cnt, cap, B, H, L, d, M, N, scale, out, c, lse, stream);
+}
 
-    if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
-    fgattn::FwdParams prm;
-    prm.kept_idx = kept_idx;
-    prm.kept_cnt = kept_cnt;
-    prm.out = static_cast<__nv_bfloat16*>(out);
-    prm.lse = lse;
-    prm.cap = kept_idx ? cap : L;
-    prm.L = L;
-    prm.QB = (L + M - 1) / M;
-    prm.items = B * H * prm.QB;
-    prm.scale_log2 = scale * 1.4426950408889634f;
-    // Lists of whole 16-key runs (N a multiple of 16) load as TMA tiles: tile layout.
-    // Anything else is gathered row by row: gather layout (more K producer warps).
-    const bool gather = kept_idx != nullptr && N % 16 != 0;
-    cudaStream_t s = (cudaStream_t)stream;
-    const int64_t rows = B * H * L;
-    if (d == 128)
-        return gather ? dispatch_m<128, true>(prm, q, k, v, rows, M, s) : dispatch_m<128, false>(prm, q, k, v, rows, M, s);
-    return gather ? dispatch_m<64, true>(prm, q, k, v, rows, M, s) : dispatch_m<64, false>(prm, q, k, v, rows, M, s);
+fgattn_status fgattn_forward_strided(const void* q, const int64_t* q_strides, const void* k, const int64_t* k_strides,
+                                     const void* v, const int64_t* v_strides, const int32_t* kept_idx,
+                                     const int32_t* kept_cnt, int64_t cap, int64_t B, int64_t H, int64_t L, int64_t d,
+                                     int64_t M, int64_t N, float scale, void* out, const int64_t* out_strides,
+                                     float* lse, fgattn_stream_t stream) {
+    if (!q_strides || !k_strides || !v_strides || !out_strides) return FGATTN_ERR_INVALID_ARG;
+    // The stride of a dimension of extent 1 is never applied: give it a valid value.
+    auto norm = [&](const int64_t* st) {
+        return Strides{{B == 1 ? d : st[0], H == 1 ? d : st[1], L == 1 ? d : st[2]}};
+    };
+    const Strides qs = norm(q_strides), ks = norm(k_strides), vs = norm(v_strides), os = norm(out_strides);
+    return forward_impl(q, qs, k, ks, v, vs, kept_idx, kept_cnt, cap, B, H, L, d, M, N, scale, out, os, lse, stream);
 }
 
 fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* bits) {

@@ -64,6 +64,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int3
 
 // Row gather: four rows y0..y3 of a one-row-high box at column x, written as four
 // consecutive box rows at dst (swizzled by the tensor map's mode).
+// Tiled TMA load of a 4-D box (x innermost), completion counted on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int32_t x, int32_t y, int32_t z,
+                                            int32_t w, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int32_t x, int32_t y0, int32_t y1,
                                             int32_t y2, int32_t y3, uint32_t bar) {
     asm volatile(

@@ -110,6 +110,27 @@ fgattn_status fgattn_forward(const void* q, const void* k, const void* v, const 
                              fgattn_stream_t stream);
 
 /*
+ * fgattn_forward on tensors in any [B][H][L][d]-indexable layout with d
+ * contiguous: [B][L][H][d] (the usual layout of a transformer's activations),
+ * q, k, v as views of one packed [B][L][3][H][d] projection, and so on.  Same
+ * operation, kept lists, lse layout ([B][H][L], contiguous) and errors as
+ * fgattn_forward; the results are identical to fgattn_forward's on the same
+ * values stored contiguously.
+ *   x_strides  in  HOST int64[3]: element strides {batch, head, token} of x;
+ *                  element (b, h, l, e) of x is x[b*s[0] + h*s[1] + l*s[2] + e].
+ * Requirements (else INVALID_ARG): every stride >= d and a multiple of 8
+ * elements (16 bytes); k and v strides multiples of d; the strides of a
+ * dimension of extent 1 are ignored.  Views of out for different (b, h, l) must
+ * not overlap.  UNSUPPORTED if the rows of k span 2^31 rows of d elements or
+ * more.
+ */
+fgattn_status fgattn_forward_strided(const void* q, const int64_t* q_strides, const void* k, const int64_t* k_strides,
+                                     const void* v, const int64_t* v_strides, const int32_t* kept_idx,
+                                     const int32_t* kept_cnt, int64_t cap, int64_t B, int64_t H, int64_t L, int64_t d,
+                                     int64_t M, int64_t N, float scale, void* out, const int64_t* out_strides,
+                                     float* lse, fgattn_stream_t stream);
+
+/*
  * Synchronise `stream`, then report (and, if clear != 0, reset) the device
  * error bits (FGATTN_DEVERR_*) recorded on the current device since the last
  * clear.  *bits may be NULL.  Returns DEVICE if any bit is set, CUDA if the

@@ -114,3 +114,44 @@ def test_compact_rejects(kw, status):
 def test_valid_call_without_gpu_reports_cuda_error():
     # All arguments valid, so the launch is attempted; with no device it fails cleanly.
     assert _cmp() == F.ERR_CUDA
+
+
+def _fwd_strided(qs=None, ks=None, vs=None, os_=None, **kw):
+    a = dict(q=P, k=P, v=P, idx=P, cnt=P, cap=64, B=2, H=4, L=64, d=128, M=64, N=16, scale=0.1, out=P, lse=P)
+    a.update(kw)
+    blhd = (a["L"] * a["H"] * a["d"], a["d"], a["H"] * a["d"])  # [B][L][H][d]
+    arr = lambda s: None if s == "null" else (ctypes.c_int64 * 3)(*(blhd if s is None else s))
+    return F._lib.fgattn_forward_strided(a["q"], arr(qs), a["k"], arr(ks), a["v"], arr(vs), a["idx"], a["cnt"],
+                                         a["cap"], a["B"], a["H"], a["L"], a["d"], a["M"], a["N"], a["scale"],
+                                         a["out"], arr(os_), a["lse"], None)
+
+
+def test_header_declares_strided_forward():
+    assert "fgattn_forward_strided" in declared_functions()
+
+
+@no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(qs="null"), F.ERR_INVALID_ARG),
+    (dict(os_="null"), F.ERR_INVALID_ARG),
+    (dict(qs=(64 * 4 * 128, 100, 4 * 128)), F.ERR_INVALID_ARG),    # head stride not a 16-byte multiple
+    (dict(qs=(64 * 4 * 128, 64, 4 * 128)), F.ERR_INVALID_ARG),     # stride below one row
+    (dict(ks=(64 * 4 * 128, 136, 4 * 136)), F.ERR_INVALID_ARG),    # k strides not whole rows
+    (dict(vs=(64 * 4 * 128, 128, 4 * 128 + 8)), F.ERR_INVALID_ARG),  # v token stride not whole rows
+    (dict(os_=(64 * 4 * 128, 128, -512)), F.ERR_INVALID_ARG),      # negative stride
+    (dict(d=96), F.ERR_UNSUPPORTED),
+    (dict(cap=63), F.ERR_CAPACITY),
+])
+def test_forward_strided_rejects(kw, status):
+    assert _fwd_strided(**kw) == status
+
+
+@no_gpu
+def test_forward_strided_valid_call_without_gpu_reports_cuda_error():
+    # [B][L][H][d] and a packed [B][L][3][H][d] projection are both accepted; the call fails
+    # only at the launch (no device here).
+    assert _fwd_strided() == F.ERR_CUDA
+    packed = (64 * 3 * 4 * 128, 128, 3 * 4 * 128)
+    assert _fwd_strided(qs=packed, ks=packed, vs=packed) == F.ERR_CUDA
+    # the stride of an extent-1 dimension is ignored
+    assert _fwd_strided(B=1, qs=(0, 128, 4 * 128)) == F.ERR_CUDA
