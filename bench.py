@@ -144,10 +144,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # traffic figure from the committed ncu summary (valid only for the same kernel source)
 # ---------------------------------------------------------------------------
-def ncu_traffic(workload, src_hash: str):
+def ncu_traffic(workload, src_hash: str, prefix: str = "fgattn_fwd"):
     if workload is None:
         return None, None
-    path = os.path.join(ROOT, "profiles", f"fgattn_fwd_{workload}.json")
+    path = os.path.join(ROOT, "profiles", f"{prefix}_{workload}.json")
     if not os.path.exists(path):
         return None, None
     with open(path) as f:
@@ -413,11 +413,20 @@ def main():
     peaks, peak_kind = load_peaks()
     achieved = flops_per_step / (fwd_ms * 1e-3) / 1e12
     from fine_grained_sparse_fgattn_b200 import _build
-    traffic, _ = ncu_traffic(profile_key(w, args), _build.kernel_hash("fwd"))
+    # 128-row query blocks (M = 128 lists, dense runs) run the query-major kernel
+    qm = args.dense or M == 128
+    gather = not args.dense and N % 16 != 0
+    strided = args.layout != "bhld"
+    if qm:
+        kname = f"fgattn_fwd_qm_kernel<{d},{str(gather).lower()},{str(strided).lower()}>"
+        traffic, _ = ncu_traffic(profile_key(w, args), _build.kernel_hash("fwd_qm"), "fgattn_fwd_qm")
+    else:
+        kname = f"fgattn_fwd_kernel<{d},{M},{str(gather).lower()},{str(strided).lower()}>"
+        traffic, _ = ncu_traffic(profile_key(w, args), _build.kernel_hash("fwd"))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                 "peak_kind": f"{peak_kind} bf16 burst",
-                "kernel": f"fgattn_fwd_kernel<{d},{M},{'false' if (args.dense or N % 16 == 0) else 'true'}>",
+                "kernel": kname,
                 "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "flops_per_launch": flops_per_step}
 

@@ -31,7 +31,9 @@ def source_hash() -> str:
 
 def kernel_hash(kernel: str) -> str:
     """Hash of the sources one kernel is built from (ties a profile to a kernel version)."""
-    files = {"fwd": ["attention_fwd.cuh", "sm100_ptx.cuh"], "compact": ["compact_mask.cuh"]}[kernel]
+    files = {"fwd": ["attention_fwd.cuh", "sm100_ptx.cuh"],
+             "fwd_qm": ["attention_fwd.cuh", "attention_fwd_qm.cuh", "sm100_ptx.cuh"],
+             "compact": ["compact_mask.cuh"]}[kernel]
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(CSRC, f), "rb") as fh:

@@ -8,6 +8,7 @@
 
 #include "fgattn.h"
 #include "attention_fwd.cuh"
+#include "attention_fwd_qm.cuh"
 #include "compact_mask.cuh"
 
 namespace {
@@ -114,10 +115,55 @@ fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const Strides& q
     return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
 }
 
+// Query-major kernel (128-row query blocks): M = 128 lists and dense runs.
+template <int D, bool GATHER, bool STRIDED>
+fgattn_status launch_qm(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
+                        const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows, cudaStream_t stream) {
+    using C = fgattn::QmCfg<D, GATHER>;
+    const int64_t L = prm.L;
+    if (STRIDED) {
+        if (!encode_4d(&prm.tmap_q, q, B, H, L, D, qs.s, C::MQ) || !encode_rows(&prm.tmap_k, k, k_rows, D, D, 1) ||
+            !encode_4d(&prm.tmap_k16, k, B, H, L, D, ks.s, 16) || !encode_4d(&prm.tmap_v16, v, B, H, L, D, vs.s, 16))
+            return FGATTN_ERR_CUDA;
+    } else {
+        const int64_t rows = B * H * L;
+        if (!encode_rows(&prm.tmap_q, q, rows, D, D, C::MQ) || !encode_rows(&prm.tmap_k, k, rows, D, D, 1) ||
+            !encode_rows(&prm.tmap_k16, k, rows, D, D, 16) || !encode_rows(&prm.tmap_v16, v, rows, D, D, 16))
+            return FGATTN_ERR_CUDA;
+    }
+    auto kernel = fgattn::fgattn_fwd_qm_kernel<D, GATHER, STRIDED>;
+    const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;  // one block per SM
+    static bool configured = false;  // per process; the attribute is per function
+    if (!configured) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return FGATTN_ERR_CUDA;
+        // setmaxnreg re-divides exactly the launch's registers: refuse any other count
+        cudaFuncAttributes attr;
+        if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FGATTN_ERR_CUDA;
+        if (attr.numRegs != (int)C::LAUNCH_REGS) return FGATTN_ERR_UNSUPPORTED;
+        configured = true;
+    }
+    const int sms = current_sms();
+    if (sms <= 0) return FGATTN_ERR_CUDA;
+    const int64_t grid = prm.items < sms ? prm.items : sms;
+    kernel<<<(unsigned)grid, C::THREADS, smem, stream>>>(prm);
+    return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
+}
+
 template <int D, bool GATHER, bool STRIDED>
 fgattn_status dispatch_m(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
                          const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows, int64_t M,
                          cudaStream_t s) {
+    // 128-row query blocks (M = 128 lists, or a dense run of any M: every key is kept,
+    // so the result does not depend on M) go to the query-major kernel.
+    if (M == 128 || prm.kept_idx == nullptr) {
+        prm.QB = (prm.L + 127) / 128;
+        prm.items = B * H * prm.QB;
+        // the query-major softmax needs a non-zero scale: a scale of magnitude below
+        // 1e-30 (log2 units) gives the same probabilities (every score maps to 2^0)
+        if (std::fabs(prm.scale_log2) < 1e-30f) prm.scale_log2 = prm.scale_log2 < 0.f ? -1e-30f : 1e-30f;
+        return launch_qm<D, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
+    }
     switch (M) {
         case 16: return launch_fwd<D, 16, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
         case 32: return launch_fwd<D, 32, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);

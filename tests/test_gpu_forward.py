@@ -78,14 +78,24 @@ def test_large_scores_rescale(oracle):
     parity_case(oracle, q, k, v, W.pack_tiles(tiles), M, N, 0.3)
 
 
-def test_dense_null_list_matches_all_ones():
-    L, d, M, N = 777, 128, 64, 16
+@pytest.mark.parametrize("M", [64, 128])
+def test_dense_null_list_matches_all_ones(oracle, M):
+    """A dense run (no lists) equals an all-ones mask.  Dense runs and M = 128 lists take
+    the query-major kernel (identical values); M = 64 lists take the key-major one
+    (same result within tolerance, both checked against the oracle)."""
+    L, d, N = 777, 128, 16
     QB, G = -(-L // M), -(-L // N)
     q, k, v = W.random_qkv(2, 2, L, d, seed=8)
     ones = W.pack_tiles(np.ones((2, 2, QB, G), bool))
     o1, l1, _, _ = run_gpu(q, k, v, ones, M, N, 0.1)
     o2, l2, _, _ = run_gpu(q, k, v, ones, M, N, 0.1, dense=True)
-    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    if M == 128:
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    blocks = list(range(2 * 2 * QB))
+    o_ref, l_ref = oracle.attention(q, k, v, ones, M, N, 0.1, blocks=blocks)
+    for o, l in ((o1, l1), (o2, l2)):
+        o_gpu, l_gpu = block_rows(o, l, blocks, 2, QB, M, L)
+        compare(o_gpu, l_gpu, o_ref, l_ref)
 
 
 @functools.lru_cache(maxsize=2)
@@ -118,9 +128,11 @@ def test_workload_sampled_blocks(oracle, name, N, sp, nblk):
     print(name, N, sp, stats)
 
 
-def test_corrupt_inputs_report_device_errors():
-    """Out-of-range indices and counts are caught by the kernel's own checks: error bits, no fault."""
-    L, d, M, N = 256, 128, 64, 8
+@pytest.mark.parametrize("M", [64, 128])
+def test_corrupt_inputs_report_device_errors(M):
+    """Out-of-range indices and counts are caught by the kernel's own checks: error bits, no fault
+    (M = 64: key-major kernel; M = 128: query-major kernel)."""
+    L, d, N = 256, 128, 8
     QB = -(-L // M)
     dev = torch.device("cuda", 0)
     q, k, v = (x.to(dev) for x in W.random_qkv(1, 1, L, d, seed=3))
@@ -129,12 +141,12 @@ def test_corrupt_inputs_report_device_errors():
     cnt = torch.full((1, 1, QB), 100, dtype=torch.int32, device=dev)
     F.device_error(clear=True)
     idx[0, 0, 1, 5] = L + 3
-    idx[0, 0, 2, 7] = -1
+    idx[0, 0, QB - 1, 7] = -1
     F.forward(q, k, v, idx, cnt, M, N)
     assert F.device_error(clear=True) & F.DEVERR_BAD_INDEX
     idx = torch.arange(cap, dtype=torch.int32, device=dev).repeat(1, 1, QB, 1)
     cnt[0, 0, 0] = 0
-    cnt[0, 0, 3] = cap + 50
+    cnt[0, 0, QB - 1] = cap + 50
     out, lse = F.forward(q, k, v, idx, cnt, M, N)
     assert F.device_error(clear=True) & F.DEVERR_BAD_COUNT
     assert F.device_error(clear=True) == 0

@@ -214,3 +214,194 @@ def test_model_catches_planted_protocol_errors(mutant):
         if caught:
             break
     assert caught, f"planted error {mutant} not detected"
+
+
+# ---------------------------------------------------------------------------
+# Query-major kernel (128-row query blocks): one softmax warpgroup, P in two
+# TMEM buffers, O reused across items behind an "O read" barrier.  Besides
+# deadlock and parity soundness, the model checks the three data hazards the
+# barriers exist for: S(g) overwriting a slot the softmax still reads, P.V(g)
+# reading a P buffer that the softmax has not finished writing or that a later
+# chunk has overwritten, the first P.V of an item overwriting O before the
+# previous item's epilogue has read it, and the epilogue reading O before the
+# item's last P.V has executed.  (The "O read" barrier turns out to be implied
+# by the softmax's own order -- the next item's first P.V needs that item's
+# first P, written after the epilogue -- and is kept as a guard.)
+# ---------------------------------------------------------------------------
+def simulate_qm(nchs, NK, rng, need_p=0.3, mutant=None):
+    KF = [Bar(f"k_full{i}") for i in range(NK)]
+    KE = [Bar(f"k_empty{i}") for i in range(NK)]
+    VF = [Bar(f"v_full{i}") for i in range(2)]
+    QF, QE = Bar("q_full"), Bar("q_empty")
+    SF = [Bar(f"s_full{i}") for i in range(2)]
+    SR = [Bar(f"s_free{i}") for i in range(2)]
+    single_p = mutant == "single_pfull"
+    PF = [Bar("p_full0")] * 2 if single_p else [Bar(f"p_full{i}") for i in range(2)]
+    OD = [Bar(f"o_done{i}") for i in range(2)]
+    OE = Bar("o_empty")
+    copies, pipe = [], []
+    stream = [(it, c, n) for it, n in enumerate(nchs) for c in range(n)]
+    G = len(stream)
+    s_reading = [None, None]  # chunk whose scores the softmax is reading from slot i
+    p_written = [None, None]  # chunk whose probabilities P buffer i holds (complete)
+    o_reading = [None]        # item whose O the epilogue is reading
+    pv_done = [0] * len(nchs)  # P.V products executed per item
+
+    def execute(op):
+        kind, g = op
+        it, c, n = stream[g]
+        if kind == "S":
+            if s_reading[g & 1] is not None:
+                raise Bug(f"S{g} overwrites slot {g & 1} while chunk {s_reading[g & 1]} is read")
+        else:  # P.V
+            if p_written[g & 1] != g:
+                raise Bug(f"PV{g} reads P buffer {g & 1} holding chunk {p_written[g & 1]}")
+            if c == 0 and o_reading[0] is not None:
+                raise Bug(f"PV{g} (first of item {it}) overwrites O while item {o_reading[0]} is read")
+            pv_done[it] += 1
+
+    def k_producer():
+        g = 0
+        for it, n in enumerate(nchs):
+            if it > 0:
+                yield from wait(QE, it - 1)
+            copies.append(QF)
+            for c in range(n):
+                gc = g + c
+                if gc >= NK:
+                    yield from wait(KE[gc % NK], gc // NK - 1)
+                copies.append(KF[gc % NK])
+                yield ("step",)
+            g += n
+
+    def v_producer():
+        for gc in range(G):
+            if gc >= 2:
+                yield from wait(OD[gc & 1], (gc - 2) >> 1)
+            copies.append(VF[gc % 2])
+            yield ("step",)
+
+    def issue_s(gc):
+        it, c, n = stream[gc]
+        if c == 0:
+            yield from wait(QF, it)
+        yield from wait(KF[gc % NK], gc // NK)
+        if gc >= 2:
+            yield from wait(SR[gc & 1], (gc >> 1) - 1)
+        pipe.append(("mma", ("S", gc)))
+        pipe.append(("commit", SF[gc & 1]))
+
+    def issue_pv(gc):
+        it, c, n = stream[gc]
+        if c == 0 and it > 0 and mutant != "no_oempty":
+            yield from wait(OE, it - 1)
+        yield from wait(VF[gc % 2], gc // 2)
+        yield from wait(PF[gc & 1], gc if single_p else gc >> 1)
+        pipe.append(("mma", ("PV", gc)))
+        pipe.append(("commit", OD[gc & 1]))
+
+    def issuer():
+        g = 0
+        for it, n in enumerate(nchs):
+            for c in range(min(n, 2)):
+                yield from issue_s(g + c)
+            for c in range(n):
+                if c + 2 < n:
+                    yield from issue_s(g + c + 2)
+                yield from issue_pv(g + c)
+            g += n
+
+    def softmax():
+        g = 0
+        for it, n in enumerate(nchs):
+            for c in range(n):
+                gc = g + c
+                yield from wait(SF[gc & 1], gc >> 1)
+                s_reading[gc & 1] = gc
+                KE[gc % NK].arrive()
+                if c == n - 1:
+                    QE.arrive()
+                yield ("step",)
+                if rng.random() < need_p and c > 0:  # rescale: O must hold chunk gc-1
+                    yield from wait(OD[(gc - 1) & 1], (gc - 1) >> 1)
+                if gc >= 2 and mutant != "no_pbuf":
+                    yield from wait(OD[(gc - 2) & 1], (gc - 2) >> 1)
+                p_written[gc & 1] = None  # being overwritten
+                yield ("step",)
+                p_written[gc & 1] = gc
+                s_reading[gc & 1] = None
+                SR[gc & 1].arrive()
+                PF[gc & 1].arrive()
+            e = g + n - 1
+            if mutant != "no_epilogue_wait":
+                yield from wait(OD[e & 1], e >> 1)
+            if pv_done[it] != n:
+                raise Bug(f"epilogue of item {it} reads O after {pv_done[it]} of {n} P.V products")
+            o_reading[0] = it
+            yield ("step",)
+            o_reading[0] = None
+            OE.arrive()
+            g += n
+
+    roles = {"K": k_producer(), "V": v_producer(), "I": issuer(), "W": softmax()}
+    state = {r: None for r in roles}
+    done = set()
+    idle_rounds = 0
+    for _ in range(500000):
+        if len(done) == len(roles):
+            return
+        progressed = False
+        if copies and rng.random() < 0.5:
+            copies.pop(rng.randrange(len(copies))).arrive()
+            progressed = True
+        if pipe and rng.random() < 0.5:
+            op = pipe.pop(0)
+            if op[0] == "commit":
+                op[1].arrive()
+            else:
+                execute(op[1])
+            progressed = True
+        order = [r for r in roles if r not in done]
+        rng.shuffle(order)
+        for r in order:
+            try:
+                y = next(roles[r])
+            except StopIteration:
+                done.add(r)
+                progressed = True
+                continue
+            if y != state[r] or y[0] != "wait":
+                progressed = True
+            state[r] = y
+        idle_rounds = 0 if (progressed or copies or pipe) else idle_rounds + 1
+        if idle_rounds > 3:
+            raise Bug(f"deadlock: {dict((r, state[r]) for r in roles if r not in done)}")
+    raise Bug("no termination")
+
+
+@pytest.mark.parametrize("NK", [2, 3, 4])
+def test_query_major_protocol_is_sound(NK):
+    for i, nchs in enumerate(CASES + _random_cases(12, NK * 17)):
+        for trial in range(6):
+            simulate_qm(nchs, NK, random.Random(trial * 7919 + i))
+
+
+def test_query_major_o_read_barrier_is_implied():
+    for i, nchs in enumerate(CASES + _random_cases(12, 99)):
+        for trial in range(6):
+            simulate_qm(nchs, 3, random.Random(trial * 13 + i), mutant="no_oempty")
+
+
+@pytest.mark.parametrize("mutant", ["no_pbuf", "no_epilogue_wait", "single_pfull"])
+def test_query_major_model_catches_planted_errors(mutant):
+    caught = False
+    for i, nchs in enumerate(CASES + _random_cases(20, 5)):
+        for trial in range(10):
+            try:
+                simulate_qm(nchs, 4, random.Random(trial * 31 + i), mutant=mutant)
+            except Bug:
+                caught = True
+                break
+        if caught:
+            break
+    assert caught, f"planted error {mutant} not detected"
