@@ -10,27 +10,30 @@
 // chunks of 128:
 //     S [128 q x 128 keys]  = Q_blk [128 x D] . K_chunk^T      (MMA1, A and B in shared memory)
 //     O [128 q x D]        += P [128 x 128 keys] . V_chunk     (MMA2, A = P in TMEM, B = V in shared memory)
-// A softmax thread owns one query row (one TMEM lane) with all 128 scores of
-// a chunk, so its running maximum is a thread-local quantity: no warpgroup
-// barrier and no cross-lane reduction per chunk.  Probabilities are taken
+// Two softmax warpgroups each take half of a chunk's keys; a softmax thread
+// owns one query row (one TMEM lane) and 64 scores of the chunk, so a row's
+// maximum needs no cross-lane reduction: the two halves combine their maxima
+// through shared memory with one barrier of the 256 softmax threads per chunk.  Probabilities are taken
 // against a reference mref that is raised only when a row maximum exceeds it
 // by more than TAU (log2 units); raising it rescales the row's partial sum and
 // its O row in TMEM (warp-collective TMEM access, so a warp rescales when any
 // of its rows needs it).  P goes back to TMEM as bf16 pairs (two buffers) and
 // feeds MMA2 directly, so P never touches shared memory.
 //
-// The softmax reads a chunk's scores twice: all 128 at once for the row
-// maximum, then 32 at a time in a rolled loop for the probabilities.  Its
-// speed follows the size of its loop body: fully unrolled passes (scores kept
-// in registers) and double-buffered loads measured 5-12 % slower, and 16-wide
-// pieces or a rolled first pass (more load round trips) 4-14 % slower.
+// Each softmax thread reads its 64 scores twice: all at once for the row
+// maximum, then 32 at a time in a rolled loop for the probabilities.  With a
+// single softmax warpgroup (128 scores per thread) the kernel measured about
+// 7 % slower; the speed follows the size of the loop body: fully unrolled
+// passes (scores kept in registers) and double-buffered loads measured 2-12 %
+// slower, and 16-wide pieces or a rolled first pass 4-14 % slower.
 //
-// Warp roles (384 threads):
-//   warps 0-3   softmax + epilogue (thread t = query row t = TMEM lane t)
-//   warp  4     TMEM allocation + single-thread tcgen05.mma issue (S of chunk c+2 before P.V of chunk c)
-//   warps 5-7   K producer: query tile (TMA), K rows (TMA boxes for 16-key runs, gather4 otherwise);
+// Warp roles (512 threads):
+//   warps 0-7   softmax + epilogue: warpgroup g = keys [64 g, 64 g + 64) of every chunk,
+//               thread t of a warpgroup = query row t = TMEM lane t
+//   warp  8     TMEM allocation + single-thread tcgen05.mma issue (S of chunk c+2 before P.V of chunk c)
+//   warps 9-11  K producer: query tile (TMA), K rows (TMA boxes for 16-key runs, gather4 otherwise);
 //               two warps for lists of 16-key runs, three for row-by-row lists
-//   warps 8-11  V producer: V rows (TMA boxes for 16-key runs, cp.async otherwise)
+//   warps 12-15 V producer: V rows (TMA boxes for 16-key runs, cp.async otherwise)
 // TMEM columns: S slots [0, 128) and [128, 256), P buffers [256, 320) and [320, 384) (bf16 pairs),
 // O [384, 384 + D).
 // Every mbarrier wait is bounded; on timeout the block records an error bit,
@@ -51,14 +54,17 @@ struct QmCfg {
     static constexpr int Q_TILE = MQ * D * 2;
     static constexpr int NV = 2;  // V slot (c % 2) is free once P.V of chunk c-2 completed
     static constexpr int LIMIT = 227 * 1024 - 1024 - 256;
-    static constexpr int MISC = 64 * 8 + 64;
+    static constexpr int XCH = 2 * 2 * 128 * 4 + 2 * 128 * 4;  // row maxima [2][2][128], row sums [2][128]
+    static constexpr int MISC = 64 * 8 + 64 + XCH;
     static constexpr int NK = (4 * KV_TILE + NV * KV_TILE + Q_TILE + MISC <= LIMIT) ? 4
                               : (3 * KV_TILE + NV * KV_TILE + Q_TILE + MISC <= LIMIT) ? 3
                                                                                       : 2;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + NK * KV_TILE;
     static constexpr int OFF_Q = OFF_V + NV * KV_TILE;
-    static constexpr int OFF_BAR = OFF_Q + Q_TILE;
+    static constexpr int OFF_XMAX = OFF_Q + Q_TILE;        // float [chunk parity][key half][row]
+    static constexpr int OFF_XSUM = OFF_XMAX + 2 * 2 * 128 * 4;  // float [key half][row]
+    static constexpr int OFF_BAR = OFF_XSUM + 2 * 128 * 4;
     // barriers: k_full[NK] k_empty[NK] v_full[NV] q_full q_empty s_full[2] s_free[2] p_full[2] o_done[2] o_empty drain
     static constexpr int B_KFULL = 0, B_KEMPTY = NK, B_VFULL = 2 * NK, B_QFULL = 2 * NK + NV, B_QEMPTY = B_QFULL + 1;
     static constexpr int B_SFULL = B_QFULL + 2, B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2;
@@ -69,15 +75,15 @@ struct QmCfg {
     static_assert(BYTES <= LIMIT, "shared memory layout");
     static constexpr int SMEM_REQUEST = BYTES + 1024;  // + alignment slack
     static constexpr uint32_t COL_S = 0, COL_P = 256, COL_O = 384, TMEM_COLS = 512;
-    static constexpr int THREADS = 384;
-    // Register split: 128 softmax threads x 232 + 256 others x 136 = 384 x 168 (the
-    // launch's allocation at 384 threads per block, one block per SM).
-    static constexpr uint32_t LAUNCH_REGS = 168, SOFT_REGS = 232, AUX_REGS = 136;
-    static_assert(128 * SOFT_REGS + 256 * AUX_REGS <= THREADS * LAUNCH_REGS, "register split");
+    static constexpr int THREADS = 512;
+    // Register split: 256 softmax threads x 160 + 256 others x 96 = 512 x 128 (the
+    // launch's allocation at 512 threads per block, one block per SM).
+    static constexpr uint32_t LAUNCH_REGS = 128, SOFT_REGS = 160, AUX_REGS = 96;
+    static_assert(256 * SOFT_REGS + 256 * AUX_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
 template <int D, bool GATHER, bool STRIDED>
-__global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_constant__ FwdParams p) {
     using C = QmCfg<D, GATHER>;
     constexpr int NK = C::NK, NV = C::NV, MQ = C::MQ;
     constexpr float TAU = 8.0f;
@@ -95,7 +101,7 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    if (warp == 4) {
+    if (warp == 8) {
         ptx::tmem_alloc(sbase + C::OFF_TMEM, C::TMEM_COLS);
         ptx::tmem_relinquish();
     }
@@ -109,12 +115,12 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
         ptx::mbar_init(BAR(C::B_QEMPTY), 1);
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(BAR(C::B_SFULL + i), 1);
-            ptx::mbar_init(BAR(C::B_SFREE + i), 128);
+            ptx::mbar_init(BAR(C::B_SFREE + i), 256);
             ptx::mbar_init(BAR(C::B_ODONE + i), 1);
         }
-        ptx::mbar_init(BAR(C::B_PFULL), 128);
-        ptx::mbar_init(BAR(C::B_PFULL + 1), 128);
-        ptx::mbar_init(BAR(C::B_OEMPTY), 128);
+        ptx::mbar_init(BAR(C::B_PFULL), 256);
+        ptx::mbar_init(BAR(C::B_PFULL + 1), 256);
+        ptx::mbar_init(BAR(C::B_OEMPTY), 256);
         ptx::mbar_init(BAR(C::B_DRAIN), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -128,10 +134,10 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
     const uint32_t tO = tmem + C::COL_O;
     const int64_t L = p.L;
 
-    if (warp >= 5 && warp < 8) {
+    if (warp >= 9 && warp < 12) {
         // ===================================================== K producer (TMA)
         ptx::regs_dec<C::AUX_REGS>();
-        const int kw = warp - 5;
+        const int kw = warp - 9;
         if (kw < C::KWARPS) {
             // segments of 16 keys per warp: 0-3 / 4-7 (two warps) or 0-2 / 3-5 / 6-7 (three);
             // four lanes (4-row groups) per segment
@@ -240,10 +246,10 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
                 bounded_wait(BAR(C::B_KFULL + (int)(i % NK)), (uint32_t)((i / NK) & 1), abort_flag, false);
             if (q_issued > 0) bounded_wait(BAR(C::B_QFULL), (uint32_t)((q_issued - 1) & 1), abort_flag, false);
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 12) {
         // ===================================================== V producer (TMA boxes / cp.async)
         ptx::regs_dec<C::AUX_REGS>();
-        const int vw = warp - 8;        // rows [32*vw, 32*vw + 32) of each chunk = two segments
+        const int vw = warp - 12;       // rows [32*vw, 32*vw + 32) of each chunk = two segments
         constexpr int PPR = D / 8;      // 16-byte pieces per row
         constexpr int RPI = 32 / PPR;   // rows per warp instruction
         int64_t g = 0;
@@ -327,7 +333,7 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
             g += nch;
         }
         ptx::cp_async_wait_all();
-    } else if (warp == 4) {
+    } else if (warp == 8) {
         // ===================================================== MMA issuer
         ptx::regs_dec<C::AUX_REGS>();
         if (lane == 0) {
@@ -394,13 +400,23 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
         }
         __syncwarp();
     } else {
-        // ===================================================== softmax + epilogue (warps 0-3)
+        // ===================================================== softmax + epilogue (warps 0-7)
+        // Two warpgroups, one per half of every chunk's keys: warpgroup g takes keys
+        // [64 g, 64 g + 64).  Both own all 128 query rows (thread t = row t = TMEM lane t),
+        // so a row's maximum is combined from the two halves once per chunk through
+        // shared memory and one barrier of the 256 threads; both halves then use the same
+        // reference.  O's columns are split between the two warpgroups for rescaling and
+        // for the epilogue; the row sum is the sum of the two halves' partial sums.
         ptx::regs_inc<C::SOFT_REGS>();
-        const int t = threadIdx.x;  // query row of the block = TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int wg = warp >> 2;          // key half
+        const int t = threadIdx.x & 127;   // query row of the block = TMEM lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
+        float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM);
         const float cs = p.scale_log2;  // never 0 (the host substitutes a tiny scale)
         // a masked key's score: scaled by cs it becomes -inf, and it never wins the row max
         const float masked = cs > 0.f ? -INFINITY : INFINITY;
+        constexpr int OH = D / 2;  // O columns per warpgroup
         int64_t g = 0;
         for (int64_t item = blockIdx.x; item < p.items; item += gridDim.x) {
             const int64_t bh = item / p.QB;
@@ -408,74 +424,79 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
             const int64_t cnt = item_count(p, item, false);
             const int64_t nch = (cnt + 127) / 128;
             float mref = -INFINITY;  // reference of this row (log2 units of the scaled scores)
-            float lsum0 = 0.f, lsum1 = 0.f;
+            float lsum = 0.f;        // this half's partial row sum
             bool failed = false;
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
                 const int s = (int)(gc & 1);
                 if (!bounded_wait(BAR(C::B_SFULL + s), (uint32_t)((gc >> 1) & 1), abort_flag)) failed = true;
                 ptx::tc_fence_after();
-                if (t == 0) {
+                if (threadIdx.x == 0) {
                     // MMA1 of this chunk has finished reading its K slot (and, for the
                     // item's last chunk, the query tile)
                     ptx::mbar_arrive(BAR(C::B_KEMPTY + (int)(gc % NK)));
                     if (c == nch - 1) ptx::mbar_arrive(BAR(C::B_QEMPTY));
                 }
-                float sc[4][32];
+                const uint32_t srow = tS + (uint32_t)s * 128u + (uint32_t)wg * 64u + lane_base;
+                const int64_t rem = cnt - c * 128 - wg * 64;  // valid keys of this half
+                // ---- this half's row maximum of the scaled scores
+                float mloc;
+                {
+                    float sc[2][32];
+                    ptx::tmem_ld32(srow, sc[0]);
+                    ptx::tmem_ld32(srow + 32, sc[1]);
+                    ptx::tmem_wait_ld();
+                    if (rem < 64) {
 #pragma unroll
-                for (int pi = 0; pi < 4; ++pi) ptx::tmem_ld32(tS + (uint32_t)s * 128u + pi * 32 + lane_base, sc[pi]);
-                ptx::tmem_wait_ld();
-                const int64_t rem = cnt - c * 128;
-                if (rem < 128) {
-#pragma unroll
-                    for (int j = 0; j < 128; ++j)
-                        if (j >= rem) sc[j / 32][j % 32] = masked;
-                }
-                // ---- row maximum of the scaled scores (thread-local)
-                float mx;
-                if (cs > 0.f) {
-                    float a = sc[0][0], b = sc[1][0], e = sc[2][0], f = sc[3][0];
-#pragma unroll
-                    for (int j = 1; j < 32; j += 2) {
-                        a = ptx::max3(a, sc[0][j], sc[0][j + 1 < 32 ? j + 1 : j]);
-                        b = ptx::max3(b, sc[1][j], sc[1][j + 1 < 32 ? j + 1 : j]);
-                        e = ptx::max3(e, sc[2][j], sc[2][j + 1 < 32 ? j + 1 : j]);
-                        f = ptx::max3(f, sc[3][j], sc[3][j + 1 < 32 ? j + 1 : j]);
+                        for (int j = 0; j < 64; ++j)
+                            if (j >= rem) sc[j / 32][j % 32] = masked;
                     }
-                    mx = fmaxf(fmaxf(a, b), fmaxf(e, f)) * cs;
-                } else {
-                    float a = sc[0][0], b = sc[1][0], e = sc[2][0], f = sc[3][0];
+                    if (cs > 0.f) {
+                        float a = sc[0][0], b = sc[1][0];
 #pragma unroll
-                    for (int j = 1; j < 32; ++j) {
-                        a = fminf(a, sc[0][j]);
-                        b = fminf(b, sc[1][j]);
-                        e = fminf(e, sc[2][j]);
-                        f = fminf(f, sc[3][j]);
+                        for (int j = 1; j < 32; j += 2) {
+                            a = ptx::max3(a, sc[0][j], sc[0][j + 1 < 32 ? j + 1 : j]);
+                            b = ptx::max3(b, sc[1][j], sc[1][j + 1 < 32 ? j + 1 : j]);
+                        }
+                        mloc = fmaxf(a, b) * cs;
+                    } else {
+                        float a = sc[0][0], b = sc[1][0];
+#pragma unroll
+                        for (int j = 1; j < 32; ++j) {
+                            a = fminf(a, sc[0][j]);
+                            b = fminf(b, sc[1][j]);
+                        }
+                        mloc = fminf(a, b) * cs;
                     }
-                    mx = fminf(fminf(a, b), fminf(e, f)) * cs;
                 }
+                // ---- combine with the other half (buffers alternate by chunk parity: a half
+                // writes parity gc & 1 again only after both passed the barrier of chunk gc+1)
+                xmax[(s * 2 + wg) * 128 + t] = mloc;
+                ptx::named_sync(1, 256);
+                const float mx = fmaxf(mloc, xmax[(s * 2 + (wg ^ 1)) * 128 + t]);  // -inf if the half is empty
                 // ---- raise the reference when the row maximum exceeds it by more than TAU
                 const bool need = mx > mref + TAU;
                 if (__any_sync(0xffffffffu, need)) {
                     const float mnew = need ? mx : mref;
                     const float alpha = ptx::ex2(mref - mnew);  // 0 on the item's first chunk, 1 for rows not raised
-                    lsum0 *= alpha;
-                    lsum1 *= alpha;
+                    lsum *= alpha;
                     if (c > 0) {
-                        // O holds this item's chunks < c: wait for the last of them, rescale the row
+                        // O holds this item's chunks < c: wait for the last of them, rescale
+                        // this warpgroup's half of the row
                         const int64_t gp = gc - 1;
                         if (!bounded_wait(BAR(C::B_ODONE + (int)(gp & 1)), (uint32_t)((gp >> 1) & 1), abort_flag))
                             failed = true;
                         ptx::tc_fence_after();
 #pragma unroll
-                        for (int pi = 0; pi < D / 32; ++pi) {
+                        for (int pi = 0; pi < OH / 32; ++pi) {
                             float o[32];
-                            ptx::tmem_ld32(tO + pi * 32 + lane_base, o);
+                            const uint32_t oa = tO + (uint32_t)(wg * OH + pi * 32) + lane_base;
+                            ptx::tmem_ld32(oa, o);
                             ptx::tmem_wait_ld();
                             uint32_t ob[32];
 #pragma unroll
                             for (int j = 0; j < 32; ++j) ob[j] = __float_as_uint(o[j] * alpha);
-                            ptx::tmem_st32(tO + pi * 32 + lane_base, ob);
+                            ptx::tmem_st32(oa, ob);
                         }
                         ptx::tmem_wait_st();
                         // the rescaled accumulator must reach TMEM before the next P.V
@@ -483,7 +504,7 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
                     }
                     mref = mnew;
                 }
-                // ---- probabilities, 32 keys at a time (the scores are read from TMEM again)
+                // ---- probabilities of this half, 32 keys at a time (scores read from TMEM again)
                 const float nm = -mref;
                 const int pbuf = (int)(gc & 1);
                 // P buffer pbuf is free once the P.V that last read it (chunk gc-2) has completed
@@ -496,11 +517,11 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
 #pragma unroll
                 for (int j = 0; j < 8; ++j) ls[j] = 0.f;
 #pragma unroll 1
-                for (int pi = 0; pi < 4; ++pi) {
+                for (int pi = 0; pi < 2; ++pi) {
                     float x[32];
-                    ptx::tmem_ld32(tS + (uint32_t)s * 128u + pi * 32 + lane_base, x);
+                    ptx::tmem_ld32(srow + pi * 32, x);
                     ptx::tmem_wait_ld();
-                    if (rem < 128) {
+                    if (rem < 64) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             if (pi * 32 + j >= rem) x[j] = masked;
@@ -515,9 +536,10 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
                         __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
                         pkf[j] = __uint_as_float(*reinterpret_cast<uint32_t*>(&h));
                     }
-                    ptx::tmem_st16(tP + (uint32_t)pbuf * 64u + pi * 16 + lane_base, pkf);
+                    // P columns: keys 2k, 2k+1 of the chunk in column k
+                    ptx::tmem_st16(tP + (uint32_t)pbuf * 64u + (uint32_t)wg * 32u + pi * 16 + lane_base, pkf);
                 }
-                lsum0 += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                lsum += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 // S slot s has been read for the last time; P of this chunk is in TMEM
@@ -527,12 +549,14 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
             // ===================== epilogue: O / l -> bf16 row, lse
             const int64_t e = g + nch - 1;
             if (!bounded_wait(BAR(C::B_ODONE + (int)(e & 1)), (uint32_t)((e >> 1) & 1), abort_flag)) failed = true;
-            if (ptx::named_red_or(1, 128, failed)) break;
+            if (ptx::named_red_or(1, 256, failed)) break;
             ptx::tc_fence_after();
-            const float l = lsum0 + lsum1;
+            xsum[wg * 128 + t] = lsum;
+            ptx::named_sync(1, 256);
+            const float l = xsum[t] + xsum[128 + t];  // the same order in both halves
             const float inv = 1.0f / l;
             const int64_t row = qb * MQ + t;
-            if (p.lse != nullptr && row < L) {
+            if (wg == 0 && p.lse != nullptr && row < L) {
                 float lg;
                 asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l));
                 p.lse[bh * L + row] = (mref + lg) * 0.69314718055994530942f;
@@ -545,9 +569,10 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
                 orow = p.out + ((size_t)bh * L + row) * D;
             }
 #pragma unroll
-            for (int pi = 0; pi < D / 32; ++pi) {
+            for (int pi = 0; pi < OH / 32; ++pi) {
+                const int col = wg * OH + pi * 32;
                 float o[32];
-                ptx::tmem_ld32(tO + pi * 32 + lane_base, o);
+                ptx::tmem_ld32(tO + (uint32_t)col + lane_base, o);
                 ptx::tmem_wait_ld();
                 if (row < L) {
 #pragma unroll
@@ -558,7 +583,7 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
                             __nv_bfloat162 h = __floats2bfloat162_rn(o[v4 * 8 + 2 * j] * inv, o[v4 * 8 + 2 * j + 1] * inv);
                             w[j] = *reinterpret_cast<uint32_t*>(&h);
                         }
-                        *reinterpret_cast<uint4*>(orow + pi * 32 + v4 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<uint4*>(orow + col + v4 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
             }
@@ -572,7 +597,7 @@ __global__ void __launch_bounds__(384, 1) fgattn_fwd_qm_kernel(const __grid_cons
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (warp == 4) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == 8) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace fgattn

@@ -49,6 +49,10 @@ FUZZ = [
     (257, 128, 64, 1, 0.4, 1), (700, 128, 64, 16, 0.3, 1), (129, 128, 128, 64, 0.5, 1), (600, 128, 128, 7, 0.25, 1),
     (200, 64, 64, 2, 0.6, 1), (513, 64, 128, 3, 0.3, 1), (640, 128, 32, 64, 0.5, 1), (1000, 128, 64, 33, 0.1, 1),
     (128, 128, 64, 128, 0.0, 1), (383, 128, 16, 1, 1.0, 1), (97, 64, 16, 100, 0.5, 1), (450, 128, 128, 1, 0.05, 2),
+    # 128-row blocks (query-major kernel): one partial block, a single key, exact multiples,
+    # keys of a chunk split unevenly between the two softmax halves
+    (100, 128, 128, 16, 0.5, 1), (1, 128, 128, 1, 1.0, 1), (256, 64, 128, 128, 0.3, 2), (384, 128, 128, 32, 0.2, 1),
+    (200, 128, 128, 5, 0.35, 1),
 ]
 
 
