@@ -22,7 +22,7 @@ import torch
 
 from . import _build
 
-__all__ = ["kept_capacity", "compact_mask", "forward", "masked_forward_noalloc", "device_error", "status_string", "num_sms",
+__all__ = ["kept_capacity", "compact_mask", "forward", "masked_forward_noalloc", "attention_from_host", "device_error", "status_string", "num_sms",
            "FgattnError", "LIB_PATH", "DEVERR_BAD_INDEX", "DEVERR_BAD_COUNT", "DEVERR_TIMEOUT"]
 
 LIB_PATH = _build.LIB
@@ -48,6 +48,9 @@ def _load() -> ctypes.CDLL:
     lib.fgattn_forward_strided.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64,
                                            ctypes.c_float, p, p, p, p]
     lib.fgattn_forward_strided.restype = i32
+    lib.fgattn_attention_from_host.argtypes = [p, p, p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64,
+                                               ctypes.c_float, p, p, p, p, i64, p]
+    lib.fgattn_attention_from_host.restype = i32
     lib.fgattn_masked_forward_noalloc.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64, ctypes.c_float, p, p, p]
     lib.fgattn_masked_forward_noalloc.restype = i32
     lib.fgattn_device_error.argtypes = [p, i32, ctypes.POINTER(ctypes.c_uint32)]
@@ -174,6 +177,58 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kept_idx: Optiona
     else:
         st = _lib.fgattn_forward(qp, kp, vp, ip, cp, cap, B, H, L, d, M, N, scale, op, lp, _stream_ptr(stream))
         _check(st, "fgattn_forward")
+    return out, lse
+
+
+def _host(t: torch.Tensor, name: str, dtypes) -> int:
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def attention_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: torch.Tensor, M: int, N: int,
+                        scale: Optional[float] = None, buffers: Optional[dict] = None, out: Optional[torch.Tensor] = None,
+                        lse: Optional[torch.Tensor] = None, heads_per_group: int = 4, device=None, stream=None):
+    """Host tensors in, host tensors out: copy-in, compaction, forward and copy-out pipelined by head groups.
+
+    q, k, v: bf16 [B,H,L,d] and mask int32/uint32 [B,H,QB,W] on the host (pinned for overlap).
+    `buffers` holds the device tensors q, k, v, mask, kept_idx, kept_cnt, out, lse (allocated here
+    when not given).  Returns (out, lse) host tensors, complete once `stream` is synchronised."""
+    B, H, L, d = q.shape
+    QB = -(-L // M)
+    cap = kept_capacity(L)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if buffers is None:
+        buffers = {"q": torch.empty(q.shape, dtype=q.dtype, device=dev),
+                   "k": torch.empty(q.shape, dtype=q.dtype, device=dev),
+                   "v": torch.empty(q.shape, dtype=q.dtype, device=dev),
+                   "mask": torch.empty(mask.shape, dtype=mask.dtype, device=dev),
+                   "kept_idx": torch.empty((B, H, QB, cap), dtype=torch.int32, device=dev),
+                   "kept_cnt": torch.empty((B, H, QB), dtype=torch.int32, device=dev),
+                   "out": torch.empty(q.shape, dtype=q.dtype, device=dev),
+                   "lse": torch.empty((B, H, L), dtype=torch.float32, device=dev)}
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, pin_memory=True)
+    bf = (torch.bfloat16,)
+    mk = (torch.int32, torch.uint32)
+    b = buffers
+    if b["kept_idx"].shape[-1] != cap:
+        raise ValueError("buffers['kept_idx'] must have a last dimension of kept_capacity(L)")
+    st = _lib.fgattn_attention_from_host(
+        _host(q, "q", bf), _host(k, "k", bf), _host(v, "v", bf), _host(mask, "mask", mk),
+        _dev(b["q"], "q buffer", bf), _dev(b["k"], "k buffer", bf), _dev(b["v"], "v buffer", bf),
+        _dev(b["mask"], "mask buffer", mk), _dev(b["kept_idx"], "kept_idx", (torch.int32,)),
+        _dev(b["kept_cnt"], "kept_cnt", (torch.int32,)), cap, B, H, L, d, M, N, scale,
+        _dev(b["out"], "out buffer", bf), _dev(b["lse"], "lse buffer", (torch.float32,)),
+        _host(out, "out", bf), _host(lse, "lse", (torch.float32,)), int(heads_per_group), _stream_ptr(stream))
+    _check(st, "fgattn_attention_from_host")
     return out, lse
 
 

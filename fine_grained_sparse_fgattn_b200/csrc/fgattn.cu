@@ -326,6 +326,125 @@ const char* fgattn_status_string(fgattn_status status) {
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
+// Host-to-host attention with the transfers overlapped with the kernels.
+//
+// The (b, h) pairs are independent, so the call splits them into groups and
+// pipelines, per group: host-to-device copies of q, k, v and the mask on one
+// internal stream, compaction + forward on the caller's stream, device-to-host
+// copies of out and lse on a second internal stream.  Events order the three;
+// group i computes while group i+1 is copied in and group i-1 is copied out.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace {
+
+constexpr int kMaxGroups = 64;
+
+struct PipeState {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, end = nullptr;
+    cudaEvent_t copied[kMaxGroups] = {}, computed[kMaxGroups] = {};
+};
+constexpr int kMaxPipeDevices = 64;
+std::mutex g_pipe_mutex;
+PipeState g_pipe[kMaxPipeDevices];
+
+// Streams and events of the current device (created on first use).  The caller
+// holds g_pipe_mutex: calls are enqueued one at a time, so every wait pairs
+// with the record of its own call.
+fgattn_status pipe_state(PipeState** st) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FGATTN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxPipeDevices) return FGATTN_ERR_UNSUPPORTED;
+    PipeState& ps = g_pipe[dev];
+    if (!ps.in) {
+        const unsigned ef = cudaEventDisableTiming;
+        if (cudaStreamCreateWithFlags(&ps.in, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&ps.out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ps.start, ef) != cudaSuccess || cudaEventCreateWithFlags(&ps.end, ef) != cudaSuccess)
+            return FGATTN_ERR_CUDA;
+        for (int i = 0; i < kMaxGroups; ++i)
+            if (cudaEventCreateWithFlags(&ps.copied[i], ef) != cudaSuccess ||
+                cudaEventCreateWithFlags(&ps.computed[i], ef) != cudaSuccess)
+                return FGATTN_ERR_CUDA;
+    }
+    *st = &ps;
+    return FGATTN_OK;
+}
+
+}  // namespace
+
+extern "C" fgattn_status fgattn_attention_from_host(
+    const void* q_host, const void* k_host, const void* v_host, const uint32_t* mask_host, void* q, void* k, void* v,
+    uint32_t* mask, int32_t* kept_idx, int32_t* kept_cnt, int64_t cap, int64_t B, int64_t H, int64_t L, int64_t d,
+    int64_t M, int64_t N, float scale, void* out, float* lse, void* out_host, float* lse_host, int64_t heads_per_group,
+    fgattn_stream_t stream) {
+    if (!q_host || !k_host || !v_host || !mask_host || !out_host) return FGATTN_ERR_INVALID_ARG;
+    if (!q || !k || !v || !mask || !kept_idx || !kept_cnt || !out) return FGATTN_ERR_INVALID_ARG;
+    if ((lse == nullptr) != (lse_host == nullptr)) return FGATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || L < 1 || M < 1 || N < 1 || d < 1 || heads_per_group < 1) return FGATTN_ERR_INVALID_ARG;
+    if (L > INT32_MAX || !std::isfinite(scale)) return FGATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kept_idx))
+        return FGATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(mask) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return FGATTN_ERR_INVALID_ARG;
+    if (cap < L || (cap & 3)) return FGATTN_ERR_CAPACITY;
+    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;
+    const int64_t BH = B * H;
+    int64_t hpg = heads_per_group;
+    if ((BH + hpg - 1) / hpg > kMaxGroups) hpg = (BH + kMaxGroups - 1) / kMaxGroups;
+    const int64_t groups = (BH + hpg - 1) / hpg;
+    const int64_t QB = (L + M - 1) / M;
+    const int64_t Ng = N > L ? L : N;
+    const int64_t W = ((L + Ng - 1) / Ng + 31) / 32;
+    const size_t row_bytes = (size_t)L * d * 2;  // one head of q, k, v or out
+
+    std::lock_guard<std::mutex> lock(g_pipe_mutex);
+    PipeState* ps = nullptr;
+    fgattn_status st = pipe_state(&ps);
+    if (st != FGATTN_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    // the copies start after everything already enqueued on the caller's stream
+    if (cudaEventRecord(ps->start, cs) != cudaSuccess || cudaStreamWaitEvent(ps->in, ps->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(ps->out, ps->start, 0) != cudaSuccess)
+        return FGATTN_ERR_CUDA;
+    auto at = [](const void* base, size_t off) { return static_cast<const char*>(base) + off; };
+    auto atw = [](void* base, size_t off) { return static_cast<char*>(base) + off; };
+    for (int64_t gi = 0; gi < groups; ++gi) {
+        const int64_t h0 = gi * hpg;
+        const int64_t hn = BH - h0 < hpg ? BH - h0 : hpg;
+        const size_t off = (size_t)h0 * row_bytes, bytes = (size_t)hn * row_bytes;
+        const size_t moff = (size_t)h0 * QB * W * 4, mbytes = (size_t)hn * QB * W * 4;
+        if (cudaMemcpyAsync(atw(q, off), at(q_host, off), bytes, cudaMemcpyHostToDevice, ps->in) != cudaSuccess ||
+            cudaMemcpyAsync(atw(k, off), at(k_host, off), bytes, cudaMemcpyHostToDevice, ps->in) != cudaSuccess ||
+            cudaMemcpyAsync(atw(v, off), at(v_host, off), bytes, cudaMemcpyHostToDevice, ps->in) != cudaSuccess ||
+            cudaMemcpyAsync(atw(mask, moff), at(mask_host, moff), mbytes, cudaMemcpyHostToDevice, ps->in) != cudaSuccess ||
+            cudaEventRecord(ps->copied[gi], ps->in) != cudaSuccess || cudaStreamWaitEvent(cs, ps->copied[gi], 0) != cudaSuccess)
+            return FGATTN_ERR_CUDA;
+        st = fgattn_compact_mask(reinterpret_cast<const uint32_t*>(atw(mask, moff)), 1, hn, L, M, N,
+                                 kept_idx + h0 * QB * cap, kept_cnt + h0 * QB, cap, stream);
+        if (st != FGATTN_OK) return st;
+        st = fgattn_forward(atw(q, off), atw(k, off), atw(v, off), kept_idx + h0 * QB * cap, kept_cnt + h0 * QB, cap, 1,
+                            hn, L, d, M, N, scale, atw(out, off), lse ? lse + h0 * L : nullptr, stream);
+        if (st != FGATTN_OK) return st;
+        if (cudaEventRecord(ps->computed[gi], cs) != cudaSuccess ||
+            cudaStreamWaitEvent(ps->out, ps->computed[gi], 0) != cudaSuccess ||
+            cudaMemcpyAsync(atw(out_host, off), at(out, off), bytes, cudaMemcpyDeviceToHost, ps->out) != cudaSuccess)
+            return FGATTN_ERR_CUDA;
+        if (lse && cudaMemcpyAsync(lse_host + h0 * L, lse + h0 * L, (size_t)hn * L * 4, cudaMemcpyDeviceToHost,
+                                   ps->out) != cudaSuccess)
+            return FGATTN_ERR_CUDA;
+    }
+    // the caller's stream is complete (host results included) once it passes this point
+    if (cudaEventRecord(ps->end, ps->out) != cudaSuccess || cudaStreamWaitEvent(cs, ps->end, 0) != cudaSuccess)
+        return FGATTN_ERR_CUDA;
+    return FGATTN_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Mask-driven forward for callers that cannot allocate device memory.
 //
 // Some callers are handed their input and output buffers and nothing else: a

@@ -9,13 +9,14 @@
  * precision; this header states the readings the library implements.
  *
  * Conventions shared by every entry point
- *   - All tensor pointers are DEVICE pointers owned by the caller.  The
- *     library allocates no device memory per call and keeps no reference to
- *     any pointer after the call returns.
+ *   - Tensor pointers are DEVICE pointers owned by the caller unless an entry
+ *     point marks them HOST.  The library allocates no device memory per call
+ *     and keeps no reference to any pointer after the call returns.
  *   - Work is enqueued on `stream` (0 = the legacy default stream) and runs
  *     asynchronously; argument validation happens synchronously on the host
  *     before anything is enqueued, and a call that returns an error status has
- *     enqueued nothing.
+ *     enqueued nothing (fgattn_attention_from_host: unless the status is CUDA,
+ *     which can leave the copies and kernels of earlier head groups enqueued).
  *   - Shapes: B batch, H heads, L tokens, d head dimension.
  *       QB = ceil(L / M) query blocks, G = ceil(L / N) key groups,
  *       W  = ceil(G / 32) mask words per query block.
@@ -137,6 +138,38 @@ fgattn_status fgattn_forward_strided(const void* q, const int64_t* q_strides, co
  * synchronisation failed, else OK.
  */
 fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* bits);
+
+/*
+ * Host to host: the whole path (copy in, compaction, forward, copy out) for
+ * inputs and results in host memory, with the transfers overlapped with the
+ * kernels.  The (b, h) pairs are split into groups of heads_per_group (at
+ * most 64 groups; more heads per group if needed); for each group the call
+ * copies q, k, v and the mask to the device on an internal stream, runs
+ * fgattn_compact_mask and fgattn_forward on `stream`, and copies out (and lse)
+ * back on a second internal stream, so that one group computes while the next
+ * is copied in and the previous one copied out.  Contiguous layouts only.
+ *   q_host, k_host, v_host  in   HOST bf16 [B][H][L][d] (pinned memory for overlap)
+ *   mask_host               in   HOST uint32 [B][H][QB][W]
+ *   q, k, v, mask           out  DEVICE buffers of the same shapes (filled by the call)
+ *   kept_idx, kept_cnt      out  DEVICE [B][H][QB][cap], [B][H][QB] (as fgattn_compact_mask)
+ *   out, lse                out  DEVICE bf16 [B][H][L][d], fp32 [B][H][L] (lse may be NULL)
+ *   out_host, lse_host      out  HOST, same shapes (lse_host NULL exactly when lse is NULL)
+ * Asynchronous with respect to the host: the host results are complete once
+ * `stream` has passed the point of the call (cudaStreamSynchronize(stream) or
+ * an event).  The copies start after all work already enqueued on `stream`.
+ * No device memory is allocated; the first call on a device creates two
+ * streams and a set of events, kept until exit.  Calls from several host
+ * threads are enqueued one at a time.
+ * Errors: as fgattn_compact_mask and fgattn_forward; INVALID_ARG also for a
+ * NULL host pointer or heads_per_group < 1.  The method of the paper has no
+ * counterpart: this is transfer scheduling around its computation.
+ */
+fgattn_status fgattn_attention_from_host(const void* q_host, const void* k_host, const void* v_host,
+                                         const uint32_t* mask_host, void* q, void* k, void* v, uint32_t* mask,
+                                         int32_t* kept_idx, int32_t* kept_cnt, int64_t cap, int64_t B, int64_t H,
+                                         int64_t L, int64_t d, int64_t M, int64_t N, float scale, void* out,
+                                         float* lse, void* out_host, float* lse_host, int64_t heads_per_group,
+                                         fgattn_stream_t stream);
 
 /*
  * Size of the kept-list scratch array that fgattn_masked_forward_noalloc

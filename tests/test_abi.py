@@ -155,3 +155,32 @@ def test_forward_strided_valid_call_without_gpu_reports_cuda_error():
     assert _fwd_strided(qs=packed, ks=packed, vs=packed) == F.ERR_CUDA
     # the stride of an extent-1 dimension is ignored
     assert _fwd_strided(B=1, qs=(0, 128, 4 * 128)) == F.ERR_CUDA
+
+
+def test_header_declares_host_pipeline():
+    assert "fgattn_attention_from_host" in declared_functions()
+
+
+def _from_host(**kw):
+    a = dict(qh=P, kh=P, vh=P, mh=P, q=P, k=P, v=P, m=P, idx=P, cnt=P, cap=64, B=1, H=4, L=64, d=128, M=64, N=16,
+             scale=0.1, out=P, lse=P, outh=P, lseh=P, hpg=2)
+    a.update(kw)
+    return F._lib.fgattn_attention_from_host(a["qh"], a["kh"], a["vh"], a["mh"], a["q"], a["k"], a["v"], a["m"],
+                                             a["idx"], a["cnt"], a["cap"], a["B"], a["H"], a["L"], a["d"], a["M"],
+                                             a["N"], a["scale"], a["out"], a["lse"], a["outh"], a["lseh"], a["hpg"],
+                                             None)
+
+
+@no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(qh=None), F.ERR_INVALID_ARG),
+    (dict(outh=None), F.ERR_INVALID_ARG),
+    (dict(lseh=None), F.ERR_INVALID_ARG),       # lse on the device but not on the host
+    (dict(hpg=0), F.ERR_INVALID_ARG),
+    (dict(idx=P + 4), F.ERR_INVALID_ARG),
+    (dict(cap=60), F.ERR_CAPACITY),
+    (dict(d=96), F.ERR_UNSUPPORTED),
+    (dict(M=48), F.ERR_UNSUPPORTED),
+])
+def test_from_host_rejects(kw, status):
+    assert _from_host(**kw) == status
