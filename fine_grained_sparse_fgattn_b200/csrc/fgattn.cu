@@ -15,6 +15,8 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+constexpr int kMaxConfigDevices = 64;
+
 // cuTensorMapEncodeTiled, fetched through the runtime so the library needs no -lcuda.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -95,8 +97,11 @@ fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const Strides& q
     // Request enough shared memory that exactly one block is resident per SM:
     // the grid is persistent (one block per SM, static round-robin over work).
     const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;
-    static bool configured = false;  // per process; the attribute is per function
-    if (!configured) {
+    // the attribute is per function and device: set and checked once per device
+    static bool configured[kMaxConfigDevices] = {};
+    int cdev = 0;
+    if (cudaGetDevice(&cdev) != cudaSuccess || cdev < 0 || cdev >= kMaxConfigDevices) return FGATTN_ERR_CUDA;
+    if (!configured[cdev]) {
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return FGATTN_ERR_CUDA;
         // The warp roles re-divide the block's registers with setmaxnreg, which only
@@ -106,7 +111,7 @@ fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const Strides& q
         if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FGATTN_ERR_CUDA;
         const bool split = C::SOFT_REGS != C::LAUNCH_REGS || C::AUX_REGS != C::LAUNCH_REGS;
         if (split && attr.numRegs != (int)C::LAUNCH_REGS) return FGATTN_ERR_UNSUPPORTED;
-        configured = true;
+        configured[cdev] = true;
     }
     const int sms = current_sms();
     if (sms <= 0) return FGATTN_ERR_CUDA;
@@ -133,15 +138,18 @@ fgattn_status launch_qm(fgattn::FwdParams& prm, const void* q, const Strides& qs
     }
     auto kernel = fgattn::fgattn_fwd_qm_kernel<D, GATHER, STRIDED>;
     const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;  // one block per SM
-    static bool configured = false;  // per process; the attribute is per function
-    if (!configured) {
+    // the attribute is per function and device: set and checked once per device
+    static bool configured[kMaxConfigDevices] = {};
+    int cdev = 0;
+    if (cudaGetDevice(&cdev) != cudaSuccess || cdev < 0 || cdev >= kMaxConfigDevices) return FGATTN_ERR_CUDA;
+    if (!configured[cdev]) {
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return FGATTN_ERR_CUDA;
         // setmaxnreg re-divides exactly the launch's registers: refuse any other count
         cudaFuncAttributes attr;
         if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FGATTN_ERR_CUDA;
         if (attr.numRegs != (int)C::LAUNCH_REGS) return FGATTN_ERR_UNSUPPORTED;
-        configured = true;
+        configured[cdev] = true;
     }
     const int sms = current_sms();
     if (sms <= 0) return FGATTN_ERR_CUDA;
