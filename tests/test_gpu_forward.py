@@ -156,3 +156,21 @@ def test_corrupt_inputs_report_device_errors(M):
     assert F.device_error(clear=True) == 0
     # the block with a clamped count of 1 attends to key 0 only
     assert torch.equal(out[0, 0, :M], v[0, 0, 0].expand(M, d))
+
+
+@pytest.mark.parametrize("M,N,d", [(64, 16, 128), (16, 3, 64), (32, 8, 128), (64, 1, 128), (128, 64, 128)])
+def test_scores_rising_far_after_the_first_chunk(oracle, M, N, d):
+    """Keys from position 400 on share a large component with every query, so their
+    scores exceed the maxima of each block's first chunk by far more than 2^32:
+    both kernels must raise their references (and rescale the partial sums and O)
+    by large steps in the middle of an item."""
+    L = 700
+    QB, G = -(-L // M), -(-L // N)
+    q, k, v = W.random_qkv(1, 2, L, d, seed=41)
+    u = torch.zeros(d)
+    u[0] = 1.0
+    late = (torch.arange(L) >= 400).float().reshape(1, 1, L, 1)
+    q = (q.float() + 4.0 * u).to(torch.bfloat16)
+    k = (k.float() + late * 120.0 * u).to(torch.bfloat16)
+    tiles = W.random_tiles(1, 2, QB, G, 0.5, seed=42)
+    parity_case(oracle, q, k, v, W.pack_tiles(tiles), M, N, 1.0 / np.sqrt(d))
