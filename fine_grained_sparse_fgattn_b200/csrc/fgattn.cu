@@ -1,10 +1,13 @@
 // C ABI of the tile-sparse attention library (declared in include/fgattn.h).
 // Host side only: argument validation, launch configuration, device error
-// word.  The kernels are in compact_mask.cuh and attention_fwd.cuh.
+// word, the host-to-host copy pipeline and the allocation-free entry point.
+// The kernels are in compact_mask.cuh, attention_fwd.cuh (key-major) and
+// attention_fwd_qm.cuh (query-major).
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "fgattn.h"
 #include "attention_fwd.cuh"
@@ -343,7 +346,6 @@ const char* fgattn_status_string(fgattn_status status) {
 // group i computes while group i+1 is copied in and group i-1 is copied out.
 // ---------------------------------------------------------------------------
 
-#include <mutex>
 
 namespace {
 
@@ -463,7 +465,6 @@ extern "C" fgattn_status fgattn_attention_from_host(
 // array that the library itself holds on every device that loads it.
 // ---------------------------------------------------------------------------
 
-#include <mutex>
 
 namespace {
 
