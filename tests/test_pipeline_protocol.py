@@ -228,36 +228,55 @@ def test_model_catches_planted_protocol_errors(mutant):
 # by the softmax's own order -- the next item's first P.V needs that item's
 # first P, written after the epilogue -- and is kept as a guard.)
 # ---------------------------------------------------------------------------
-def simulate_qm(nchs, NK, rng, need_p=0.3, mutant=None):
+class Rendezvous:
+    """A named barrier among `n` roles: each instance (key) completes when all arrived."""
+
+    def __init__(self, n):
+        self.n, self.count = n, {}
+
+
+def rendezvous(rv, key):
+    rv.count[key] = rv.count.get(key, 0) + 1
+    while rv.count[key] < rv.n:
+        yield ("barrier", key)
+
+
+def simulate_qm(nchs, NK, rng, need_p=0.3, mutant=None, halves=1):
+    """halves = 2: two softmax warpgroups, each taking half of every chunk's keys
+    (counts of two on the softmax barriers, a rendezvous per chunk to combine the
+    row maxima and one per item before the epilogue)."""
     KF = [Bar(f"k_full{i}") for i in range(NK)]
     KE = [Bar(f"k_empty{i}") for i in range(NK)]
     VF = [Bar(f"v_full{i}") for i in range(2)]
     QF, QE = Bar("q_full"), Bar("q_empty")
     SF = [Bar(f"s_full{i}") for i in range(2)]
-    SR = [Bar(f"s_free{i}") for i in range(2)]
+    SR = [Bar(f"s_free{i}", halves) for i in range(2)]
     single_p = mutant == "single_pfull"
-    PF = [Bar("p_full0")] * 2 if single_p else [Bar(f"p_full{i}") for i in range(2)]
+    pcount = 1 if mutant == "pfull_count1" else halves
+    PF = [Bar("p_full0", pcount)] * 2 if single_p else [Bar(f"p_full{i}", pcount) for i in range(2)]
     OD = [Bar(f"o_done{i}") for i in range(2)]
-    OE = Bar("o_empty")
+    OE = Bar("o_empty", halves)
+    RV = Rendezvous(halves)
     copies, pipe = [], []
     stream = [(it, c, n) for it, n in enumerate(nchs) for c in range(n)]
     G = len(stream)
-    s_reading = [None, None]  # chunk whose scores the softmax is reading from slot i
-    p_written = [None, None]  # chunk whose probabilities P buffer i holds (complete)
-    o_reading = [None]        # item whose O the epilogue is reading
-    pv_done = [0] * len(nchs)  # P.V products executed per item
+    need = [rng.random() < need_p for _ in range(G)]  # reference raised (the same in both halves)
+    s_reading = [set(), set()]  # halves still reading the scores of slot i
+    p_written = [{}, {}]        # P buffer i: half -> chunk whose probabilities it holds (complete)
+    o_reading = set()           # (item, half) of epilogues reading O
+    pv_done = [0] * len(nchs)   # P.V products executed per item
 
     def execute(op):
         kind, g = op
         it, c, n = stream[g]
         if kind == "S":
-            if s_reading[g & 1] is not None:
-                raise Bug(f"S{g} overwrites slot {g & 1} while chunk {s_reading[g & 1]} is read")
+            if s_reading[g & 1]:
+                raise Bug(f"S{g} overwrites slot {g & 1} while halves {s_reading[g & 1]} read it")
         else:  # P.V
-            if p_written[g & 1] != g:
-                raise Bug(f"PV{g} reads P buffer {g & 1} holding chunk {p_written[g & 1]}")
-            if c == 0 and o_reading[0] is not None:
-                raise Bug(f"PV{g} (first of item {it}) overwrites O while item {o_reading[0]} is read")
+            if any(p_written[g & 1].get(h) != g for h in range(halves)):
+                raise Bug(f"PV{g} reads P buffer {g & 1} holding {p_written[g & 1]}")
+            if c == 0 and o_reading:
+                raise Bug(f"PV{g} (first of item {it}) overwrites O while {o_reading} read it")
             pv_done[it] += 1
 
     def k_producer():
@@ -311,25 +330,28 @@ def simulate_qm(nchs, NK, rng, need_p=0.3, mutant=None):
                 yield from issue_pv(g + c)
             g += n
 
-    def softmax():
+    def softmax(h):
         g = 0
         for it, n in enumerate(nchs):
             for c in range(n):
                 gc = g + c
                 yield from wait(SF[gc & 1], gc >> 1)
-                s_reading[gc & 1] = gc
-                KE[gc % NK].arrive()
-                if c == n - 1:
-                    QE.arrive()
+                s_reading[gc & 1].add(h)
+                if h == 0:
+                    KE[gc % NK].arrive()
+                    if c == n - 1:
+                        QE.arrive()
                 yield ("step",)
-                if rng.random() < need_p and c > 0:  # rescale: O must hold chunk gc-1
+                if halves > 1:
+                    yield from rendezvous(RV, ("max", gc))
+                if need[gc] and c > 0:  # rescale: O must hold chunk gc-1
                     yield from wait(OD[(gc - 1) & 1], (gc - 1) >> 1)
                 if gc >= 2 and mutant != "no_pbuf":
                     yield from wait(OD[(gc - 2) & 1], (gc - 2) >> 1)
-                p_written[gc & 1] = None  # being overwritten
+                p_written[gc & 1].pop(h, None)  # being overwritten
                 yield ("step",)
-                p_written[gc & 1] = gc
-                s_reading[gc & 1] = None
+                p_written[gc & 1][h] = gc
+                s_reading[gc & 1].discard(h)
                 SR[gc & 1].arrive()
                 PF[gc & 1].arrive()
             e = g + n - 1
@@ -337,13 +359,17 @@ def simulate_qm(nchs, NK, rng, need_p=0.3, mutant=None):
                 yield from wait(OD[e & 1], e >> 1)
             if pv_done[it] != n:
                 raise Bug(f"epilogue of item {it} reads O after {pv_done[it]} of {n} P.V products")
-            o_reading[0] = it
+            if halves > 1:
+                yield from rendezvous(RV, ("epilogue", it))
+            o_reading.add((it, h))
             yield ("step",)
-            o_reading[0] = None
+            o_reading.discard((it, h))
             OE.arrive()
             g += n
 
-    roles = {"K": k_producer(), "V": v_producer(), "I": issuer(), "W": softmax()}
+    roles = {"K": k_producer(), "V": v_producer(), "I": issuer()}
+    for h in range(halves):
+        roles[f"W{h}"] = softmax(h)
     state = {r: None for r in roles}
     done = set()
     idle_rounds = 0
@@ -370,7 +396,7 @@ def simulate_qm(nchs, NK, rng, need_p=0.3, mutant=None):
                 done.add(r)
                 progressed = True
                 continue
-            if y != state[r] or y[0] != "wait":
+            if y != state[r] or y[0] not in ("wait", "barrier"):
                 progressed = True
             state[r] = y
         idle_rounds = 0 if (progressed or copies or pipe) else idle_rounds + 1
@@ -379,26 +405,29 @@ def simulate_qm(nchs, NK, rng, need_p=0.3, mutant=None):
     raise Bug("no termination")
 
 
+@pytest.mark.parametrize("halves", [1, 2])
 @pytest.mark.parametrize("NK", [2, 3, 4])
-def test_query_major_protocol_is_sound(NK):
+def test_query_major_protocol_is_sound(NK, halves):
     for i, nchs in enumerate(CASES + _random_cases(12, NK * 17)):
         for trial in range(6):
-            simulate_qm(nchs, NK, random.Random(trial * 7919 + i))
+            simulate_qm(nchs, NK, random.Random(trial * 7919 + i), halves=halves)
 
 
-def test_query_major_o_read_barrier_is_implied():
+@pytest.mark.parametrize("halves", [1, 2])
+def test_query_major_o_read_barrier_is_implied(halves):
     for i, nchs in enumerate(CASES + _random_cases(12, 99)):
         for trial in range(6):
-            simulate_qm(nchs, 3, random.Random(trial * 13 + i), mutant="no_oempty")
+            simulate_qm(nchs, 3, random.Random(trial * 13 + i), mutant="no_oempty", halves=halves)
 
 
-@pytest.mark.parametrize("mutant", ["no_pbuf", "no_epilogue_wait", "single_pfull"])
-def test_query_major_model_catches_planted_errors(mutant):
+@pytest.mark.parametrize("mutant,halves", [("no_pbuf", 1), ("no_epilogue_wait", 1), ("single_pfull", 1),
+                                           ("no_pbuf", 2), ("pfull_count1", 2)])
+def test_query_major_model_catches_planted_errors(mutant, halves):
     caught = False
     for i, nchs in enumerate(CASES + _random_cases(20, 5)):
         for trial in range(10):
             try:
-                simulate_qm(nchs, 4, random.Random(trial * 31 + i), mutant=mutant)
+                simulate_qm(nchs, 4, random.Random(trial * 31 + i), mutant=mutant, halves=halves)
             except Bug:
                 caught = True
                 break
