@@ -184,3 +184,16 @@ def _from_host(**kw):
 ])
 def test_from_host_rejects(kw, status):
     assert _from_host(**kw) == status
+
+
+def test_binding_refuses_host_tensors():
+    """There is no CPU path: host tensors are refused before any library call."""
+    q = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        F.forward(q, q, q, None, None, 16, 16)
+    with pytest.raises(ValueError):
+        F.forward(q.transpose(1, 2), q.transpose(1, 2), q.transpose(1, 2), None, None, 16, 16)
+    with pytest.raises(ValueError):
+        F.compact_mask(torch.zeros(1, 1, 1, 1, dtype=torch.int32), 1, 1, 16, 16, 16)
+    with pytest.raises(ValueError):
+        F.masked_forward_noalloc(q, q, q, torch.zeros(1, 1, 1, 1, dtype=torch.int32), 16, 16)
