@@ -64,3 +64,14 @@ def test_lowrank_component_peaks_scores():
     q, k, _ = W.make_qkv(w, 0)
     s = (q[0, 0].float() @ k[0, 0].float().T) * w.scale
     assert s.diagonal().mean() > s.mean() + 5.0
+
+
+@pytest.mark.parametrize("N", [1, 4, 16, 64])
+def test_granularity_sweep_targets(N):
+    """The sweep regenerates the same mask family per tile width at one score sparsity,
+    with every row's own key kept."""
+    w = W.get("gransweep").with_(N=N)
+    tiles = W.make_tiles(w, 0, heads=range(1))
+    assert abs(W.score_sparsity(tiles, w) - w.sparsity) < 1e-3
+    i = np.arange(w.L)
+    assert tiles[:, :, i // w.M, i // w.N].all()
