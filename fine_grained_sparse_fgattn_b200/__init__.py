@@ -95,6 +95,21 @@ def _dev(t: torch.Tensor, name: str, dtypes) -> int:
     return t.data_ptr()
 
 
+def _geometry(L: int, M: int, N: int) -> Tuple[int, int]:
+    """(QB, W): query blocks and mask words per block (the C ABI's layout)."""
+    QB = -(-L // M)
+    G = -(-L // min(N, L))
+    return QB, -(-G // 32)
+
+
+def _numel(t: torch.Tensor, n: int, name: str) -> None:
+    """The C ABI takes plain pointers and cannot see extents: check them here."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a tensor")
+    if t.numel() != n:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {n}")
+
+
 def _dev_rows(t: torch.Tensor, name: str):
     """A [B, H, L, d] bf16 view whose last dimension is contiguous: (pointer, host int64[3] strides)."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
@@ -120,8 +135,15 @@ def compact_mask(mask: torch.Tensor, B: int, H: int, L: int, M: int, N: int,
                  kept_idx: Optional[torch.Tensor] = None, kept_cnt: Optional[torch.Tensor] = None,
                  cap: Optional[int] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Packed tile mask uint32/int32 [B,H,QB,W] -> (kept_idx int32 [B,H,QB,cap], kept_cnt int32 [B,H,QB])."""
-    QB = -(-L // M)
+    QB = -(-L // M) if M >= 1 else 0
     cap = kept_capacity(L) if cap is None else int(cap)
+    if min(B, H, L, M, N) >= 1:
+        QB, W = _geometry(L, M, N)
+        _numel(mask, B * H * QB * W, "mask")
+        if kept_idx is not None:
+            _numel(kept_idx, B * H * QB * cap, "kept_idx")
+        if kept_cnt is not None:
+            _numel(kept_cnt, B * H * QB, "kept_cnt")
     dev = mask.device
     if kept_idx is None:
         kept_idx = torch.empty((B, H, QB, cap), dtype=torch.int32, device=dev)
@@ -154,6 +176,14 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kept_idx: Optiona
         raise ValueError("out must have the shape of q")
     if lse is None and want_lse:
         lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _numel(lse, B * H * L, "lse")
+    if kept_idx is not None and min(L, M, N) >= 1:
+        QB = _geometry(L, M, N)[0]
+        if kept_idx.dim() < 1 or kept_idx.shape[-1] < L:
+            raise ValueError("kept_idx must be [B, H, QB, cap] with cap >= L")
+        _numel(kept_idx, B * H * QB * kept_idx.shape[-1], "kept_idx")
+        _numel(kept_cnt, B * H * QB, "kept_cnt")
     lp = _dev(lse, "lse", (torch.float32,)) if lse is not None else None
     strided = not all(t.is_contiguous() for t in (q, k, v, out))
     if strided:
@@ -199,8 +229,25 @@ def attention_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask:
     `buffers` holds the device tensors q, k, v, mask, kept_idx, kept_cnt, out, lse (allocated here
     when not given).  Returns (out, lse) host tensors, complete once `stream` is synchronised."""
     B, H, L, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, H, L, d] shape")
     QB = -(-L // M)
     cap = kept_capacity(L)
+    if min(L, M, N) >= 1:
+        QB, W = _geometry(L, M, N)
+        _numel(mask, B * H * QB * W, "mask")
+        if buffers is not None:
+            for name in ("q", "k", "v", "out"):
+                if buffers[name].shape != q.shape:
+                    raise ValueError(f"buffers['{name}'] must have the shape of q")
+            _numel(buffers["mask"], B * H * QB * W, "buffers['mask']")
+            _numel(buffers["kept_idx"], B * H * QB * cap, "buffers['kept_idx']")
+            _numel(buffers["kept_cnt"], B * H * QB, "buffers['kept_cnt']")
+            _numel(buffers["lse"], B * H * L, "buffers['lse']")
+        if out is not None and out.shape != q.shape:
+            raise ValueError("out must have the shape of q")
+        if lse is not None:
+            _numel(lse, B * H * L, "lse")
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     if buffers is None:
@@ -242,11 +289,19 @@ def masked_forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ma
     FGATTN_NOALLOC_SCRATCH_BYTES; larger problems raise FgattnError CAPACITY).
     Calls that can overlap on the GPU share that array and race."""
     B, H, L, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, H, L, d] shape")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if min(L, M, N) >= 1:
+        QB, W = _geometry(L, M, N)
+        _numel(mask, B * H * QB * W, "mask")
     if out is None:
         out = torch.empty_like(q)
+    if out.shape != q.shape:
+        raise ValueError("out must have the shape of q")
     if lse is None:
         lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _numel(lse, B * H * L, "lse")
     bf = (torch.bfloat16,)
     st = _lib.fgattn_masked_forward_noalloc(_dev(q, "q", bf), _dev(k, "k", bf), _dev(v, "v", bf),
                                             _dev(mask, "mask", (torch.int32, torch.uint32)), B, H, L, d, M, N,

@@ -197,3 +197,25 @@ def test_binding_refuses_host_tensors():
         F.compact_mask(torch.zeros(1, 1, 1, 1, dtype=torch.int32), 1, 1, 16, 16, 16)
     with pytest.raises(ValueError):
         F.masked_forward_noalloc(q, q, q, torch.zeros(1, 1, 1, 1, dtype=torch.int32), 16, 16)
+
+
+def test_binding_checks_extents():
+    """The C ABI cannot see buffer extents; the binding refuses wrong ones before any call."""
+    q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
+    good_mask = torch.zeros(1, 1, 4, 1, dtype=torch.int32)  # L 64, M 16 -> QB 4; N 16 -> G 4 -> W 1
+    with pytest.raises(ValueError, match="mask"):
+        F.compact_mask(torch.zeros(1, 1, 4, 2, dtype=torch.int32), 1, 1, 64, 16, 16)
+    with pytest.raises(ValueError, match="kept_idx"):
+        F.compact_mask(good_mask, 1, 1, 64, 16, 16, kept_idx=torch.zeros(1, 1, 3, 64, dtype=torch.int32))
+    with pytest.raises(ValueError, match="kept_cnt"):
+        F.forward(q, q, q, torch.zeros(1, 1, 4, 64, dtype=torch.int32), torch.zeros(1, 1, 3, dtype=torch.int32),
+                  16, 16)
+    with pytest.raises(ValueError, match="cap >= L"):
+        F.forward(q, q, q, torch.zeros(1, 1, 4, 32, dtype=torch.int32), torch.zeros(1, 1, 4, dtype=torch.int32),
+                  16, 16)
+    with pytest.raises(ValueError, match="lse"):
+        F.forward(q, q, q, None, None, 16, 16, lse=torch.zeros(1, 1, 63))
+    with pytest.raises(ValueError, match="mask"):
+        F.masked_forward_noalloc(q, q, q, torch.zeros(1, 1, 5, 1, dtype=torch.int32), 16, 16)
+    with pytest.raises(ValueError, match="mask"):
+        F.attention_from_host(q, q, q, torch.zeros(1, 1, 4, 2, dtype=torch.int32), 16, 16)
