@@ -82,7 +82,24 @@ def _check(status: int, where: str) -> None:
 
 def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
     s = torch.cuda.current_stream() if stream is None else stream
+    if stream is not None:
+        _require_current_device([("stream", s.device.index)])
     return int(s.cuda_stream)
+
+
+def _current_device() -> int:
+    return torch.cuda.current_device()
+
+
+def _require_current_device(named_indices) -> None:
+    """The C ABI launches on the current device and cannot see where a pointer lives:
+    every device tensor of a call must be on the current device (a pointer into another
+    GPU's memory would reach the kernels as an invalid address)."""
+    cur = _current_device()
+    for name, index in named_indices:
+        if index != cur:
+            raise ValueError(f"{name} is on cuda:{index} but the current device is cuda:{cur}; "
+                             f"call under torch.cuda.device({index}) or move the tensor")
 
 
 def _dev(t: torch.Tensor, name: str, dtypes) -> int:
@@ -92,6 +109,7 @@ def _dev(t: torch.Tensor, name: str, dtypes) -> int:
         raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    _require_current_device([(name, t.device.index)])
     return t.data_ptr()
 
 
@@ -118,6 +136,7 @@ def _dev_rows(t: torch.Tensor, name: str):
         raise ValueError(f"{name} has dtype {t.dtype}, expected torch.bfloat16")
     if t.dim() != 4 or (t.shape[-1] > 1 and t.stride(-1) != 1):
         raise ValueError(f"{name} must be a [B, H, L, d] view with a contiguous last dimension")
+    _require_current_device([(name, t.device.index)])
     st = (ctypes.c_int64 * 3)(*t.stride()[:3])
     return t.data_ptr(), st
 

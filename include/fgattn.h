@@ -173,7 +173,15 @@ fgattn_status fgattn_attention_from_host(const void* q_host, const void* k_host,
 
 /*
  * Size of the kept-list scratch array that fgattn_masked_forward_noalloc
- * uses: 64 MiB, held on every device that loads the library, until exit.
+ * uses: 64 MiB on every device the library is used on, held until exit.
+ * The array belongs to the library's device code, so it is reserved when that
+ * code is loaded onto a device: at the first call into the library on that
+ * device, whichever entry point it is (with lazy module loading; at context
+ * creation otherwise).  Every user of the library pays these 64 MiB per
+ * device.  A caller that cannot allocate should make one call (any entry
+ * point, e.g. fgattn_compact_mask on a tiny mask) before its allocator
+ * reserves the device's memory; if the reservation fails, every entry point
+ * returns FGATTN_ERR_CUDA.
  */
 #define FGATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
 
@@ -197,7 +205,10 @@ fgattn_status fgattn_attention_from_host(const void* q_host, const void* k_host,
  * No cudaMalloc, cudaFree or other allocating call is made.
  * Set-up: the first call on a device looks up that device's address of the
  * array (with the device current); make that first call before any stream
- * capture begins.
+ * capture begins.  The address is kept for the life of the process, so the
+ * library must not be used across a reset of that device (cudaDeviceReset or
+ * any other teardown of its primary context): after one, the kept address
+ * would no longer be the array's.
  * Sharing: every call on a device uses the same array, and it keeps the last
  * call's lists.  Calls in one stream are ordered and safe; calls that can run
  * at the same time on the GPU (different streams, no ordering between them)

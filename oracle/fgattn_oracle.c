@@ -19,7 +19,8 @@
  *   out_i = sum_j exp(s_ij - m_i) v_j / l_i
  *   lse_i = m_i + ln l_i                         (natural logarithm)
  *
- * Readings where the page is silent (each listed in the design notes):
+ * Readings where the page is silent (the CUDA library takes the same ones,
+ * written separately):
  *   - mask layout: uint32 words, tile (qb, g) is bit (g % 32) of word g / 32 of
  *     row (b, h, qb); W = ceil(G / 32) words per row; bits >= G are ignored;
  *   - the "diagonal" tiles a query block always keeps are the tiles that hold

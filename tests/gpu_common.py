@@ -69,13 +69,18 @@ def compare(o_gpu, l_gpu, o_ref, l_ref):
     return stats
 
 
-def sample_blocks(B, H, QB, n_random, seed):
-    """First block, the ragged last block of the first and of the last head, plus seeded random blocks."""
+def sample_blocks(B, H, QB, n_random, seed, whole_heads=()):
+    """First block, the ragged last block of the first and of the last head, at least
+    n_random further distinct seeded blocks, and every block of the flat heads
+    (b*H + h) listed in whole_heads."""
     rng = np.random.default_rng(seed)
     total = B * H * QB
-    chosen = {0, QB - 1, total - 1, total - QB}
-    chosen.update(int(x) for x in rng.integers(0, total, size=n_random))
-    return sorted(chosen)
+    fixed = {0, QB - 1, total - 1, total - QB}
+    for bh in whole_heads:
+        fixed.update(range(bh * QB, (bh + 1) * QB))
+    pool = np.setdiff1d(np.arange(total), np.fromiter(fixed, dtype=np.int64))
+    extra = rng.choice(pool, size=min(n_random, pool.size), replace=False)
+    return sorted(fixed | {int(x) for x in extra})
 
 
 def parity_case(oracle, q, k, v, mask_np, M, N, scale, blocks=None, dense=False):

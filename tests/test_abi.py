@@ -219,3 +219,15 @@ def test_binding_checks_extents():
         F.masked_forward_noalloc(q, q, q, torch.zeros(1, 1, 5, 1, dtype=torch.int32), 16, 16)
     with pytest.raises(ValueError, match="mask"):
         F.attention_from_host(q, q, q, torch.zeros(1, 1, 4, 2, dtype=torch.int32), 16, 16)
+
+
+def test_tensors_on_another_device_are_refused(monkeypatch):
+    """The C ABI launches on the current device and cannot tell which GPU a pointer
+    belongs to, so the binding refuses any device tensor (or stream) that is not on the
+    current device, before a pointer reaches the library."""
+    monkeypatch.setattr(F, "_current_device", lambda: 0)
+    F._require_current_device([("q", 0), ("k", 0)])
+    with pytest.raises(ValueError, match="cuda:1"):
+        F._require_current_device([("q", 0), ("k", 1)])
+    with pytest.raises(ValueError, match="stream"):
+        F._require_current_device([("stream", 2)])

@@ -20,7 +20,7 @@ import torch
 
 import fine_grained_sparse_fgattn_b200 as F
 import workloads as W
-from gpu_common import LSE_MAX_ABS, OUT_MAX_ABS, OUT_REL_RMS
+from gpu_common import LSE_MAX_ABS, OUT_MAX_ABS
 
 pytestmark = pytest.mark.gpu
 
@@ -46,14 +46,20 @@ def _case(q, k, v, mask_np, M, N):
     lse = torch.full((B, H, L), float("nan"), dtype=torch.float32, device=dev)
     assert _noalloc(qd, kd, vd, md, M, N, scale, out, lse) == F.OK
     assert F.device_error() == 0
-    return out.float().cpu().numpy(), lse.cpu().numpy(), o_ref.float().cpu().numpy(), l_ref.cpu().numpy()
+    return out, lse, o_ref, l_ref
 
 
 def _check(o, l, o_ref, l_ref):
-    assert np.isfinite(o).all() and np.isfinite(l).all()
+    # Both paths run the same kernels on the same lists, so the results must be
+    # identical bit for bit: a list read that reached a stale entry of an earlier
+    # call would change some output, however slightly.
+    assert torch.isfinite(o.float()).all() and torch.isfinite(l).all()
+    assert torch.equal(o, o_ref)
+    assert torch.equal(l, l_ref)
+    # and the usual tolerances hold trivially (kept as a readable statement of the bar)
+    o, o_ref = o.float().cpu().numpy(), o_ref.float().cpu().numpy()
     assert np.abs(o - o_ref).max() <= OUT_MAX_ABS
-    assert np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref) <= OUT_REL_RMS
-    assert np.abs(l - l_ref).max() <= LSE_MAX_ABS
+    assert np.abs(l.cpu().numpy() - l_ref.cpu().numpy()).max() <= LSE_MAX_ABS
 
 
 def test_noalloc_matches_two_call_path_twice_in_a_row():
