@@ -12,6 +12,10 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfgattn.so")
 STAMP = LIB + ".srchash"
+# Microbenchmarks of the rooflines (row loads from L2, tcgen05 issue rate, MUFU):
+# a separate library; the attention path never loads it.
+PROBES_SRC = os.path.join(CSRC, "probes", "probes.cu")
+PROBES_LIB = os.path.join(PKG, "libfgattn_probes.so")
 
 
 def _sources():
@@ -70,5 +74,24 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def _probe_deps():
+    return [PROBES_SRC] + [os.path.join(CSRC, f) for f in ("attention_fwd.cuh", "sm100_ptx.cuh")]
+
+
+def build_probes(force: bool = False, verbose: bool = False) -> str:
+    if not force and os.path.exists(PROBES_LIB) and \
+            os.path.getmtime(PROBES_LIB) >= max(os.path.getmtime(f) for f in _probe_deps()):
+        return PROBES_LIB
+    tmp = PROBES_LIB + f".tmp{os.getpid()}"
+    cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
+           "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, PROBES_SRC, "-o", tmp]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, PROBES_LIB)
+    return PROBES_LIB
+
+
 if __name__ == "__main__":
     print(build(force=True, verbose=True))
+    print(build_probes(force=True))

@@ -76,7 +76,9 @@ struct alignas(64) FwdParams {
     CUtensorMap tmap_q;    // q tiles: box {64, MQ} (contiguous) or {64, MQ, 1, 1} (strided), 128B swizzle
     CUtensorMap tmap_k;    // k rows of D elements, box {64, 1} (row gathers)
     CUtensorMap tmap_k16;  // k tiles: box {64, 16} or {64, 16, 1, 1} (16 consecutive keys)
-    CUtensorMap tmap_v16;  // same for V
+    CUtensorMap tmap_v16;  // same for V (at D = 96 the box at column 64 is half outside: zero fill)
+    // D = 96 only: columns 64..95 of q and k, 32-column boxes with 64B swizzle
+    CUtensorMap tmap_q_hi, tmap_k_hi, tmap_k16_hi;
     const __nv_bfloat16* v_base;  // V rows, gathered with cp.async where not consecutive
     // strided layout only
     int64_t k_ub, k_uh;  // k batch / head strides in rows of D elements
@@ -95,20 +97,63 @@ struct alignas(64) FwdParams {
     float scale_log2;  // scale * log2(e)
 };
 
+// UMMA shared-memory descriptor (sm_100): start address >> 4 (bits 0-13), leading
+// byte offset >> 4 (16-29), stride byte offset >> 4 (32-45), version 1 (bit 46),
+// swizzle mode (bits 61-63: 2 = 128B, 4 = 64B, 6 = 32B), built as two halves.  The
+// high half is a compile-time constant per operand; the low half moves by adding
+// (byte offset >> 4), which never carries out of the 14-bit address field for
+// shared-memory offsets below 256 KB.
+__host__ __device__ constexpr uint32_t umma_desc_hi(uint32_t sbo, uint32_t layout) {
+    return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (layout << 29);
+}
+__device__ __forceinline__ uint32_t umma_desc_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t umma_desc_join(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
+
+// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Head dimensions D in {64, 96, 128}.  Q and K rows sit in shared memory as
+// 64-column panels with 128-byte rows (128B swizzle); at D = 96 the second panel
+// holds the last 32 columns in 64-byte rows (64B swizzle), so every load stays
+// inside the rows and the score product runs D / 16 k-steps.  V rows always sit
+// in 64-column 128B-swizzled panels; at D = 96 columns 96..127 of the second
+// panel are zero, so the P.V product runs on V padded to DP = 128 columns (the
+// only shape tcgen05 offers for that operand: M = D must be 64 or 128 in the
+// key-major product), and the padded output columns are never stored.
+template <int D>
+struct HeadDim {
+    static_assert(D == 64 || D == 96 || D == 128, "head dim");
+    static constexpr int DP = D == 96 ? 128 : D;  // padded width of V, O and the shared-memory slots
+    static constexpr int KP = (D + 63) / 64;      // panels of Q and K
+    static constexpr bool NARROW = D == 96;       // second Q/K panel: 32 columns, 64B swizzle
+    __host__ __device__ static constexpr uint32_t pitch(int pn) { return (NARROW && pn == 1) ? 64u : 128u; }
+    // high word of the UMMA descriptor of Q/K panel pn (K-major; SBO = 8 rows)
+    __host__ __device__ static constexpr uint32_t desc_hi(int pn) {
+        return (NARROW && pn == 1) ? umma_desc_hi(8u * 64u, 4u) : umma_desc_hi(8u * 128u, 2u);
+    }
+};
+
 template <int D, int MQ, bool GATHER>
 struct FwdCfg {
-    static_assert(D == 64 || D == 128, "head dim");
+    using HD = HeadDim<D>;
+    static constexpr int DP = HD::DP;
     static_assert(MQ == 16 || MQ == 32 || MQ == 64 || MQ == 128, "query block");
     static constexpr int KC = 128;              // keys per chunk = MMA1 M
     static constexpr int NSW = (!GATHER && (MQ == 32 || MQ == 64)) ? 4 : 2;  // softmax warpgroups
     static constexpr int KWARPS = GATHER ? 3 : 2;                            // K producer warps
     static constexpr int CW = MQ / NSW;         // query columns per softmax warpgroup
-    static constexpr int KV_TILE = KC * D * 2;  // bytes of a K or V chunk
+    static constexpr int KV_TILE = KC * DP * 2;  // bytes of a K or V chunk slot
     static constexpr int P_ROW = (MQ * 2 < 128) ? MQ * 2 : 128;  // bytes per key row of a P panel
     static constexpr int P_CPR = P_ROW / 16;    // 16-byte chunks per P row
     static constexpr int P_PANEL = KC * P_ROW;  // bytes per P panel
     static constexpr int P_TILE = KC * MQ * 2;
-    static constexpr int Q_TILE = MQ * D * 2;
+    static constexpr int Q_TILE = MQ * DP * 2;  // query tile slot
+    static constexpr int Q_TX = MQ * D * 2;     // bytes a query-tile load delivers
     static constexpr int SROWS = (CW < 8) ? CW : (NSW == 4 ? 8 : (CW < 16 ? CW : 16));  // staging rows per group
     static constexpr int STAGE = SROWS * D * 2;
     static constexpr int MISC = NSW * (3 * CW + 4 * CW) * 4 + 64 * 8 + 64;  // mref/alpha/lfin/red, barriers
@@ -163,26 +208,6 @@ struct FwdCfg {
     static constexpr uint32_t AUX_REGS = NSW == 4 ? 64 : (MQ == 128 ? 80 : 128);
     static_assert(NSW * 128 * SOFT_REGS + 256 * AUX_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
-
-// UMMA shared-memory descriptor (sm_100): start address >> 4 (bits 0-13), leading
-// byte offset >> 4 (16-29), stride byte offset >> 4 (32-45), version 1 (bit 46),
-// swizzle mode (bits 61-63: 2 = 128B, 4 = 64B, 6 = 32B), built as two halves.  The
-// high half is a compile-time constant per operand; the low half moves by adding
-// (byte offset >> 4), which never carries out of the 14-bit address field for
-// shared-memory offsets below 256 KB.
-__host__ __device__ constexpr uint32_t umma_desc_hi(uint32_t sbo, uint32_t layout) {
-    return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (layout << 29);
-}
-__device__ __forceinline__ uint32_t umma_desc_lo(uint32_t saddr, uint32_t lbo) {
-    return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
-}
-__device__ __forceinline__ uint64_t umma_desc_join(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
-
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
 
 // Byte offset of 16-byte chunk `c` of row `r` in a swizzled panel with `row_bytes`
 // per row (128, 64 or 32): the chunk index is XORed with the row's position in
@@ -354,15 +379,17 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                     break;
                 }
                 if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(BAR(C::B_QFULL), (uint32_t)C::Q_TILE);
+                    ptx::mbar_arrive_expect_tx(BAR(C::B_QFULL), (uint32_t)C::Q_TX);
 #pragma unroll
-                    for (int pn = 0; pn < D / 64; ++pn)
+                    for (int pn = 0; pn < C::HD::KP; ++pn) {
+                        const CUtensorMap* qm = (C::HD::NARROW && pn == 1) ? &p.tmap_q_hi : &p.tmap_q;
                         if constexpr (STRIDED)
-                            ptx::tma_load_4d(QTILE + (uint32_t)pn * (MQ * 128), &p.tmap_q, pn * 64,
-                                             (int32_t)(qb * MQ), hi, bi, BAR(C::B_QFULL));
+                            ptx::tma_load_4d(QTILE + (uint32_t)pn * (MQ * 128), qm, pn * 64, (int32_t)(qb * MQ), hi,
+                                             bi, BAR(C::B_QFULL));
                         else
-                            ptx::tma_load_2d(QTILE + (uint32_t)pn * (MQ * 128), &p.tmap_q, pn * 64,
+                            ptx::tma_load_2d(QTILE + (uint32_t)pn * (MQ * 128), qm, pn * 64,
                                              (int32_t)(bh * L + qb * MQ), BAR(C::B_QFULL));
+                    }
                 }
                 ++q_issued;
                 __syncwarp();
@@ -396,25 +423,29 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                     ptx::mbar_arrive_expect_tx(BAR(C::B_KFULL + st), (uint32_t)(nseg * 16 * D * 2));
                 __syncwarp();
                 if (issuer) {
-                    const uint32_t dst = KSLOT(st) + (uint32_t)g4 * 512u;
+                    // this lane's 4 rows in panel pn (rows of pitch(pn) bytes)
+                    auto dst = [&](int pn) {
+                        return KSLOT(st) + (uint32_t)pn * (128 * 128) + (uint32_t)g4 * 4u * C::HD::pitch(pn);
+                    };
                     if (seg_run) {
                         if ((lane & 3) == 0) {
 #pragma unroll
-                            for (int pn = 0; pn < D / 64; ++pn)
+                            for (int pn = 0; pn < C::HD::KP; ++pn) {
+                                const CUtensorMap* km = (C::HD::NARROW && pn == 1) ? &p.tmap_k16_hi : &p.tmap_k16;
                                 if constexpr (STRIDED)
-                                    ptx::tma_load_4d(dst + (uint32_t)pn * (128 * 128), &p.tmap_k16, pn * 64, first,
-                                                     hi, bi, BAR(C::B_KFULL + st));
+                                    ptx::tma_load_4d(dst(pn), km, pn * 64, first, hi, bi, BAR(C::B_KFULL + st));
                                 else
-                                    ptx::tma_load_2d(dst + (uint32_t)pn * (128 * 128), &p.tmap_k16, pn * 64,
-                                                     (int32_t)(bh * L + first), BAR(C::B_KFULL + st));
+                                    ptx::tma_load_2d(dst(pn), km, pn * 64, (int32_t)(bh * L + first),
+                                                     BAR(C::B_KFULL + st));
+                            }
                         }
                     } else {
                         int32_t rows[4];
                         rows_of<STRIDED>(p, cur, krow0, true, rows);
 #pragma unroll
-                        for (int pn = 0; pn < D / 64; ++pn)
-                            ptx::tma_gather4(dst + (uint32_t)pn * (128 * 128), &p.tmap_k, pn * 64, rows[0], rows[1],
-                                             rows[2], rows[3], BAR(C::B_KFULL + st));
+                        for (int pn = 0; pn < C::HD::KP; ++pn)
+                            ptx::tma_gather4(dst(pn), (C::HD::NARROW && pn == 1) ? &p.tmap_k_hi : &p.tmap_k, pn * 64,
+                                             rows[0], rows[1], rows[2], rows[3], BAR(C::B_KFULL + st));
                     }
                 }
                 ++issued;
@@ -430,7 +461,8 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
         // ===================================================== V producer (TMA boxes / cp.async)
         if constexpr (C::AUX_REGS != C::LAUNCH_REGS) ptx::regs_dec<C::AUX_REGS>();
         const int vw = warp - (AW + 4);  // rows [32*vw, 32*vw + 32) of each chunk = two segments
-        constexpr int PPR = D / 8;     // 16-byte pieces per row
+        constexpr int DP = C::DP;
+        constexpr int PPR = DP / 8;    // 16-byte pieces per row of a V slot (padding pieces zero-filled)
         constexpr int RPI = 32 / PPR;  // rows per warp instruction
         int64_t g = 0;
         bool ok = true;
@@ -481,9 +513,10 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                     if (((runs >> (16 * sg)) & 0xFFFFu) == 0xFFFFu) {
                         const int32_t fs = __shfl_sync(0xffffffffu, first, 16 * sg);
                         if (lane == 0) {
-                            ptx::mbar_expect_tx(BAR(C::B_VFULL + st), (uint32_t)(16 * D * 2));
+                            // whole boxes, including the zero-filled columns past D
+                            ptx::mbar_expect_tx(BAR(C::B_VFULL + st), (uint32_t)(16 * DP * 2));
 #pragma unroll
-                            for (int pn = 0; pn < D / 64; ++pn) {
+                            for (int pn = 0; pn < DP / 64; ++pn) {
                                 if constexpr (STRIDED)
                                     ptx::tma_load_4d(vdst + (uint32_t)pn * (128 * 128) + (uint32_t)r0 * 128u,
                                                      &p.tmap_v16, pn * 64, fs, hi, bi, BAR(C::B_VFULL + st));
@@ -499,12 +532,16 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                             const int pc = lane % PPR;
                             const int32_t ridx = __shfl_sync(0xffffffffu, idx, rl);
                             const int r = vw * 32 + rl;
+                            // pieces past D (D = 96) are zero-filled: no bytes read from the row start
+                            const bool real = pc * 8 < D;
+                            const int pe = real ? pc * 8 : 0;
                             const __nv_bfloat16* src;
                             if constexpr (STRIDED)
-                                src = p.v_base + (size_t)(uint32_t)(vrow0 + ridx * p.v_ul) * D + pc * 8;
+                                src = p.v_base + (size_t)(uint32_t)(vrow0 + ridx * p.v_ul) * D + pe;
                             else
-                                src = vb + (size_t)ridx * D + pc * 8;
-                            ptx::cp_async_16(vdst + (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128), src, 16u);
+                                src = vb + (size_t)ridx * D + pe;
+                            ptx::cp_async_16(vdst + (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128), src,
+                                             real ? 16u : 0u);
                         }
                     }
                 }
@@ -523,9 +560,8 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
         if constexpr (C::AUX_REGS != C::LAUNCH_REGS) ptx::regs_dec<C::AUX_REGS>();
         if (lane == 0) {
             constexpr uint32_t IDESC1 = umma_idesc_bf16(128, MQ, false, false);
-            constexpr uint32_t IDESC2 = umma_idesc_bf16(D, MQ, true, true);
+            constexpr uint32_t IDESC2 = umma_idesc_bf16(C::DP, MQ, true, true);
             constexpr uint32_t P_LAYOUT = (C::P_ROW == 128) ? 2u : (C::P_ROW == 64) ? 4u : 6u;
-            constexpr uint32_t HI_KQ = umma_desc_hi(1024u, 2u);  // K rows and Q rows: K-major, 128B swizzle
             constexpr uint32_t HI_V = umma_desc_hi(1024u, 2u);   // V^T: MN-major, 128B swizzle
             constexpr uint32_t HI_P = umma_desc_hi(8u * C::P_ROW, P_LAYOUT);
             const uint32_t qlo = umma_desc_lo(QTILE, 16u);
@@ -567,8 +603,9 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
                     const uint32_t qoff = (uint32_t)(kk / 4) * (MQ * 128) + (uint32_t)(kk % 4) * 32u;
-                    const uint64_t ad = umma_desc_join(alo + (koff >> 4), HI_KQ);
-                    const uint64_t bd = umma_desc_join(qlo + (qoff >> 4), HI_KQ);
+                    // K rows and Q rows: K-major, the panel's swizzle
+                    const uint64_t ad = umma_desc_join(alo + (koff >> 4), C::HD::desc_hi(kk / 4));
+                    const uint64_t bd = umma_desc_join(qlo + (qoff >> 4), C::HD::desc_hi(kk / 4));
                     ptx::mma_bf16_ss(dS, ad, bd, IDESC1, kk > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(BAR(C::B_SFULL + s));
@@ -607,7 +644,8 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         const uint32_t col0 = (uint32_t)(wg * CW);  // this group's first query column
         // d index held by this thread in the O^T accumulator (M = D layout)
-        const int dt = (D == 128) ? t : ((lane < 16) ? wq * 16 + lane : -1);
+        // (the O^T accumulator has DP lanes; at D = 96 lanes 96..127 hold the zero padding)
+        const int dt = (C::DP == 128) ? (t < D ? t : -1) : ((lane < 16) ? wq * 16 + lane : -1);
         float* mref = reinterpret_cast<float*>(smem + C::OFF_MREF) + wg * CW;
         float* alpha = reinterpret_cast<float*>(smem + C::OFF_ALPHA) + wg * CW;
         float* lfin = reinterpret_cast<float*>(smem + C::OFF_LFIN) + wg * CW;

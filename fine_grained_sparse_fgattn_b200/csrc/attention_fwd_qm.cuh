@@ -35,7 +35,7 @@
 //               two warps for lists of 16-key runs, three for row-by-row lists
 //   warps 12-15 V producer: V rows (TMA boxes for 16-key runs, cp.async otherwise)
 // TMEM columns: S slots [0, 128) and [128, 256), P buffers [256, 320) and [320, 384) (bf16 pairs),
-// O [384, 384 + D).
+// O [384, 384 + DP) (DP = D, or 128 at D = 96: zero-padded V columns).
 // Every mbarrier wait is bounded; on timeout the block records an error bit,
 // drains its copies and MMAs, frees TMEM and exits (as fgattn_fwd_kernel).
 #pragma once
@@ -46,12 +46,14 @@ namespace fgattn {
 
 template <int D, bool GATHER>
 struct QmCfg {
-    static_assert(D == 64 || D == 128, "head dim");
+    using HD = HeadDim<D>;  // panels of Q/K, V and O padded to DP columns at D = 96
+    static constexpr int DP = HD::DP;
     static constexpr int MQ = 128;              // query rows per block = MMA M
     static constexpr int KC = 128;              // keys per chunk = MMA1 N
     static constexpr int KWARPS = GATHER ? 3 : 2;
-    static constexpr int KV_TILE = KC * D * 2;  // bytes of a K or V chunk
-    static constexpr int Q_TILE = MQ * D * 2;
+    static constexpr int KV_TILE = KC * DP * 2;  // bytes of a K or V chunk slot
+    static constexpr int Q_TILE = MQ * DP * 2;   // query tile slot
+    static constexpr int Q_TX = MQ * D * 2;      // bytes a query-tile load delivers
     static constexpr int NV = 2;  // V slot (c % 2) is free once P.V of chunk c-2 completed
     static constexpr int LIMIT = 227 * 1024 - 1024 - 256;
     static constexpr int XCH = 2 * 2 * 128 * 4 + 2 * 128 * 4;  // row maxima [2][2][128], row sums [2][128]
@@ -170,14 +172,15 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                         break;
                     }
                     if (lane == 0) {
-                        ptx::mbar_arrive_expect_tx(BAR(C::B_QFULL), (uint32_t)C::Q_TILE);
+                        ptx::mbar_arrive_expect_tx(BAR(C::B_QFULL), (uint32_t)C::Q_TX);
 #pragma unroll
-                        for (int pn = 0; pn < D / 64; ++pn) {
+                        for (int pn = 0; pn < C::HD::KP; ++pn) {
+                            const CUtensorMap* qm = (C::HD::NARROW && pn == 1) ? &p.tmap_q_hi : &p.tmap_q;
                             if constexpr (STRIDED)
-                                ptx::tma_load_4d(QTILE + (uint32_t)pn * (MQ * 128), &p.tmap_q, pn * 64,
-                                                 (int32_t)(qb * MQ), hi, bi, BAR(C::B_QFULL));
+                                ptx::tma_load_4d(QTILE + (uint32_t)pn * (MQ * 128), qm, pn * 64, (int32_t)(qb * MQ),
+                                                 hi, bi, BAR(C::B_QFULL));
                             else
-                                ptx::tma_load_2d(QTILE + (uint32_t)pn * (MQ * 128), &p.tmap_q, pn * 64,
+                                ptx::tma_load_2d(QTILE + (uint32_t)pn * (MQ * 128), qm, pn * 64,
                                                  (int32_t)(bh * L + qb * MQ), BAR(C::B_QFULL));
                         }
                     }
@@ -215,26 +218,29 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                         ptx::mbar_arrive_expect_tx(BAR(C::B_KFULL + st), (uint32_t)(nseg * 16 * D * 2));
                     __syncwarp();
                     if (issuer) {
-                        const uint32_t dst = KSLOT(st) + (uint32_t)g4 * 512u;
+                        // this lane's 4 rows in panel pn (rows of pitch(pn) bytes)
+                        auto dst = [&](int pn) {
+                            return KSLOT(st) + (uint32_t)pn * (128 * 128) + (uint32_t)g4 * 4u * C::HD::pitch(pn);
+                        };
                         if (seg_run) {
                             if ((lane & 3) == 0) {
 #pragma unroll
-                                for (int pn = 0; pn < D / 64; ++pn) {
+                                for (int pn = 0; pn < C::HD::KP; ++pn) {
+                                    const CUtensorMap* km = (C::HD::NARROW && pn == 1) ? &p.tmap_k16_hi : &p.tmap_k16;
                                     if constexpr (STRIDED)
-                                        ptx::tma_load_4d(dst + (uint32_t)pn * (128 * 128), &p.tmap_k16, pn * 64,
-                                                         first, hi, bi, BAR(C::B_KFULL + st));
+                                        ptx::tma_load_4d(dst(pn), km, pn * 64, first, hi, bi, BAR(C::B_KFULL + st));
                                     else
-                                        ptx::tma_load_2d(dst + (uint32_t)pn * (128 * 128), &p.tmap_k16, pn * 64,
-                                                         (int32_t)(bh * L + first), BAR(C::B_KFULL + st));
+                                        ptx::tma_load_2d(dst(pn), km, pn * 64, (int32_t)(bh * L + first),
+                                                         BAR(C::B_KFULL + st));
                                 }
                             }
                         } else {
                             int32_t rows[4];
                             rows_of<STRIDED>(p, cur, krow0, true, rows);
 #pragma unroll
-                            for (int pn = 0; pn < D / 64; ++pn)
-                                ptx::tma_gather4(dst + (uint32_t)pn * (128 * 128), &p.tmap_k, pn * 64, rows[0],
-                                                 rows[1], rows[2], rows[3], BAR(C::B_KFULL + st));
+                            for (int pn = 0; pn < C::HD::KP; ++pn)
+                                ptx::tma_gather4(dst(pn), (C::HD::NARROW && pn == 1) ? &p.tmap_k_hi : &p.tmap_k,
+                                                 pn * 64, rows[0], rows[1], rows[2], rows[3], BAR(C::B_KFULL + st));
                         }
                     }
                     ++issued;
@@ -250,7 +256,8 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
         // ===================================================== V producer (TMA boxes / cp.async)
         ptx::regs_dec<C::AUX_REGS>();
         const int vw = warp - 12;       // rows [32*vw, 32*vw + 32) of each chunk = two segments
-        constexpr int PPR = D / 8;      // 16-byte pieces per row
+        constexpr int DP = C::DP;
+        constexpr int PPR = DP / 8;     // 16-byte pieces per row of a V slot (padding pieces zero-filled)
         constexpr int RPI = 32 / PPR;   // rows per warp instruction
         int64_t g = 0;
         bool ok = true;
@@ -300,9 +307,10 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                     if (((runs >> (16 * sg)) & 0xFFFFu) == 0xFFFFu) {
                         const int32_t fs = __shfl_sync(0xffffffffu, first, 16 * sg);
                         if (lane == 0) {
-                            ptx::mbar_expect_tx(BAR(C::B_VFULL + st), (uint32_t)(16 * D * 2));
+                            // whole boxes, including the zero-filled columns past D
+                            ptx::mbar_expect_tx(BAR(C::B_VFULL + st), (uint32_t)(16 * DP * 2));
 #pragma unroll
-                            for (int pn = 0; pn < D / 64; ++pn) {
+                            for (int pn = 0; pn < DP / 64; ++pn) {
                                 if constexpr (STRIDED)
                                     ptx::tma_load_4d(vdst + (uint32_t)pn * (128 * 128) + (uint32_t)r0 * 128u,
                                                      &p.tmap_v16, pn * 64, fs, hi, bi, BAR(C::B_VFULL + st));
@@ -319,12 +327,16 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                             const int pc = lane % PPR;
                             const int32_t ridx = __shfl_sync(0xffffffffu, idx, rl);
                             const int r = vw * 32 + rl;
+                            // pieces past D (D = 96) are zero-filled: no bytes read from the row start
+                            const bool real = pc * 8 < D;
+                            const int pe = real ? pc * 8 : 0;
                             const __nv_bfloat16* src;
                             if constexpr (STRIDED)
-                                src = p.v_base + (size_t)(uint32_t)(vrow0 + ridx * p.v_ul) * D + pc * 8;
+                                src = p.v_base + (size_t)(uint32_t)(vrow0 + ridx * p.v_ul) * D + pe;
                             else
-                                src = vb + (size_t)ridx * D + pc * 8;
-                            ptx::cp_async_16(vdst + (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128), src, 16u);
+                                src = vb + (size_t)ridx * D + pe;
+                            ptx::cp_async_16(vdst + (uint32_t)(pc / 8) * (128 * 128) + swz(r, pc % 8, 128), src,
+                                             real ? 16u : 0u);
                         }
                     }
                 }
@@ -338,8 +350,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
         ptx::regs_dec<C::AUX_REGS>();
         if (lane == 0) {
             constexpr uint32_t IDESC1 = umma_idesc_bf16(128, 128, false, false);  // S = Q . K^T
-            constexpr uint32_t IDESC2 = umma_idesc_bf16(128, D, false, true);     // O += P . V, V N-major
-            constexpr uint32_t HI_KQ = umma_desc_hi(1024u, 2u);  // Q and K rows: K-major, 128B swizzle
+            constexpr uint32_t IDESC2 = umma_idesc_bf16(128, C::DP, false, true);  // O += P . V, V N-major
             constexpr uint32_t HI_V = umma_desc_hi(1024u, 2u);   // V rows: N-major, 128B swizzle
             const uint32_t qlo = umma_desc_lo(QTILE, 16u);
             bool ok = true;
@@ -355,10 +366,11 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                 const uint32_t dS = tS + (uint32_t)s * 128u;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    // Q tile and K chunk share one layout: 64-column panels of 128 rows x 128 B
+                    // Q tile and K chunk share one layout: 64-column panels of 128 rows (K-major, the
+                    // panel's swizzle)
                     const uint32_t off = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
-                    const uint64_t ad = umma_desc_join(qlo + (off >> 4), HI_KQ);
-                    const uint64_t bd = umma_desc_join(klo + (off >> 4), HI_KQ);
+                    const uint64_t ad = umma_desc_join(qlo + (off >> 4), C::HD::desc_hi(kk / 4));
+                    const uint64_t bd = umma_desc_join(klo + (off >> 4), C::HD::desc_hi(kk / 4));
                     ptx::mma_bf16_ss(dS, ad, bd, IDESC1, kk > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(BAR(C::B_SFULL + s));
@@ -416,7 +428,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
         const float cs = p.scale_log2;  // never 0 (the host substitutes a tiny scale)
         // a masked key's score: scaled by cs it becomes -inf, and it never wins the row max
         const float masked = cs > 0.f ? -INFINITY : INFINITY;
-        constexpr int OH = D / 2;  // O columns per warpgroup
+        constexpr int OH = C::DP / 2;  // O columns per warpgroup (padding columns included)
         int64_t g = 0;
         for (int64_t item = blockIdx.x; item < p.items; item += gridDim.x) {
             const int64_t bh = item / p.QB;
@@ -571,6 +583,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
 #pragma unroll
             for (int pi = 0; pi < OH / 32; ++pi) {
                 const int col = wg * OH + pi * 32;
+                if (col >= D) continue;  // zero padding of V (D = 96)
                 float o[32];
                 ptx::tmem_ld32(tO + (uint32_t)col + lane_base, o);
                 ptx::tmem_wait_ld();

@@ -38,32 +38,42 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 rows of d elements, `row_stride` elements apart, viewed in boxes of 64 columns x
-// box_rows rows, 128B swizzle.
-bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t d, int64_t row_stride, uint32_t box_rows) {
+// Box shapes: 64 columns with 128B swizzle (128-byte shared-memory rows), or -- for
+// columns 64..95 of a 96-element head -- 32 columns with 64B swizzle (64-byte rows).
+struct BoxCols {
+    uint32_t cols;
+    CUtensorMapSwizzle swizzle;
+};
+constexpr BoxCols kWide = {64u, CU_TENSOR_MAP_SWIZZLE_128B};
+constexpr BoxCols kNarrow = {32u, CU_TENSOR_MAP_SWIZZLE_64B};
+
+// bf16 rows of d elements, `row_stride` elements apart, viewed in boxes of bc.cols
+// columns x box_rows rows.
+bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t d, int64_t row_stride, uint32_t box_rows,
+                 BoxCols bc = kWide) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
-    const cuuint32_t box[2] = {64u, box_rows};
+    const cuuint32_t box[2] = {bc.cols, box_rows};
     const cuuint32_t estr[2] = {1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, bc.swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // [B][H][L][d] view with element strides st = {sb, sh, sl} (d contiguous) as a 4-D
-// map {d, L, H, B} in boxes of 64 columns x box_rows consecutive L positions, 128B swizzle.
+// map {d, L, H, B} in boxes of bc.cols columns x box_rows consecutive L positions.
 bool encode_4d(CUtensorMap* m, const void* base, int64_t B, int64_t H, int64_t L, int64_t d, const int64_t* st,
-               uint32_t box_rows) {
+               uint32_t box_rows, BoxCols bc = kWide) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)H, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
-    const cuuint32_t box[4] = {64u, box_rows, 1u, 1u};
+    const cuuint32_t box[4] = {bc.cols, box_rows, 1u, 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, bc.swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -80,22 +90,40 @@ int current_sms() {
     return sms;
 }
 
+// The tensor maps of one launch: query tiles of mq rows, k row gathers, 16-key k and v
+// boxes; at d = 96 also the 32-column maps of columns 64..95 of q and k.
+template <bool STRIDED>
+bool encode_maps(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
+                 const void* v, const Strides& vs, int64_t B, int64_t H, int64_t d, int64_t k_rows, uint32_t mq) {
+    const int64_t L = prm.L;
+    const bool narrow = d == 96;
+    if (STRIDED) {
+        if (!encode_4d(&prm.tmap_q, q, B, H, L, d, qs.s, mq) || !encode_rows(&prm.tmap_k, k, k_rows, d, d, 1) ||
+            !encode_4d(&prm.tmap_k16, k, B, H, L, d, ks.s, 16) || !encode_4d(&prm.tmap_v16, v, B, H, L, d, vs.s, 16))
+            return false;
+        if (narrow && (!encode_4d(&prm.tmap_q_hi, q, B, H, L, d, qs.s, mq, kNarrow) ||
+                       !encode_rows(&prm.tmap_k_hi, k, k_rows, d, d, 1, kNarrow) ||
+                       !encode_4d(&prm.tmap_k16_hi, k, B, H, L, d, ks.s, 16, kNarrow)))
+            return false;
+    } else {
+        const int64_t rows = B * H * L;
+        if (!encode_rows(&prm.tmap_q, q, rows, d, d, mq) || !encode_rows(&prm.tmap_k, k, rows, d, d, 1) ||
+            !encode_rows(&prm.tmap_k16, k, rows, d, d, 16) || !encode_rows(&prm.tmap_v16, v, rows, d, d, 16))
+            return false;
+        if (narrow && (!encode_rows(&prm.tmap_q_hi, q, rows, d, d, mq, kNarrow) ||
+                       !encode_rows(&prm.tmap_k_hi, k, rows, d, d, 1, kNarrow) ||
+                       !encode_rows(&prm.tmap_k16_hi, k, rows, d, d, 16, kNarrow)))
+            return false;
+    }
+    return true;
+}
+
 template <int D, int MQ, bool GATHER, bool STRIDED>
 fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
                          const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows,
                          cudaStream_t stream) {
     using C = fgattn::FwdCfg<D, MQ, GATHER>;
-    const int64_t L = prm.L;
-    if (STRIDED) {
-        if (!encode_4d(&prm.tmap_q, q, B, H, L, D, qs.s, MQ) || !encode_rows(&prm.tmap_k, k, k_rows, D, D, 1) ||
-            !encode_4d(&prm.tmap_k16, k, B, H, L, D, ks.s, 16) || !encode_4d(&prm.tmap_v16, v, B, H, L, D, vs.s, 16))
-            return FGATTN_ERR_CUDA;
-    } else {
-        const int64_t rows = B * H * L;
-        if (!encode_rows(&prm.tmap_q, q, rows, D, D, MQ) || !encode_rows(&prm.tmap_k, k, rows, D, D, 1) ||
-            !encode_rows(&prm.tmap_k16, k, rows, D, D, 16) || !encode_rows(&prm.tmap_v16, v, rows, D, D, 16))
-            return FGATTN_ERR_CUDA;
-    }
+    if (!encode_maps<STRIDED>(prm, q, qs, k, ks, v, vs, B, H, D, k_rows, MQ)) return FGATTN_ERR_CUDA;
     auto kernel = fgattn::fgattn_fwd_kernel<D, MQ, GATHER, STRIDED>;
     // Request enough shared memory that exactly one block is resident per SM:
     // the grid is persistent (one block per SM, static round-robin over work).
@@ -128,17 +156,7 @@ template <int D, bool GATHER, bool STRIDED>
 fgattn_status launch_qm(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
                         const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows, cudaStream_t stream) {
     using C = fgattn::QmCfg<D, GATHER>;
-    const int64_t L = prm.L;
-    if (STRIDED) {
-        if (!encode_4d(&prm.tmap_q, q, B, H, L, D, qs.s, C::MQ) || !encode_rows(&prm.tmap_k, k, k_rows, D, D, 1) ||
-            !encode_4d(&prm.tmap_k16, k, B, H, L, D, ks.s, 16) || !encode_4d(&prm.tmap_v16, v, B, H, L, D, vs.s, 16))
-            return FGATTN_ERR_CUDA;
-    } else {
-        const int64_t rows = B * H * L;
-        if (!encode_rows(&prm.tmap_q, q, rows, D, D, C::MQ) || !encode_rows(&prm.tmap_k, k, rows, D, D, 1) ||
-            !encode_rows(&prm.tmap_k16, k, rows, D, D, 16) || !encode_rows(&prm.tmap_v16, v, rows, D, D, 16))
-            return FGATTN_ERR_CUDA;
-    }
+    if (!encode_maps<STRIDED>(prm, q, qs, k, ks, v, vs, B, H, D, k_rows, C::MQ)) return FGATTN_ERR_CUDA;
     auto kernel = fgattn::fgattn_fwd_qm_kernel<D, GATHER, STRIDED>;
     const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;  // one block per SM
     // the attribute is per function and device: set and checked once per device
@@ -190,6 +208,9 @@ fgattn_status dispatch(fgattn::FwdParams& prm, const void* q, const Strides& qs,
     if (d == 128)
         return gather ? dispatch_m<128, true, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
                       : dispatch_m<128, false, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
+    if (d == 96)
+        return gather ? dispatch_m<96, true, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
+                      : dispatch_m<96, false, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
     return gather ? dispatch_m<64, true, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
                   : dispatch_m<64, false, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
 }
@@ -208,7 +229,7 @@ fgattn_status forward_impl(const void* q, const Strides& qs, const void* k, cons
     if (kept_idx && !aligned16(kept_idx)) return FGATTN_ERR_INVALID_ARG;  // rows are read as int4
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FGATTN_ERR_INVALID_ARG;
     if (kept_idx && (cap < L || (cap & 3))) return FGATTN_ERR_CAPACITY;
-    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 96 && d != 128) return FGATTN_ERR_UNSUPPORTED;
     if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
     // Strides: at least one row (d) and 16-byte multiples (TMA, vector stores); k and v
     // strides whole rows of d, so every key row is a row of the gather map over k.
@@ -400,7 +421,7 @@ extern "C" fgattn_status fgattn_attention_from_host(
     if ((reinterpret_cast<uintptr_t>(mask) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return FGATTN_ERR_INVALID_ARG;
     if (cap < L || (cap & 3)) return FGATTN_ERR_CAPACITY;
-    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 96 && d != 128) return FGATTN_ERR_UNSUPPORTED;
     if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
     if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;
     const int64_t BH = B * H;
@@ -508,7 +529,7 @@ extern "C" fgattn_status fgattn_masked_forward_noalloc(const void* q, const void
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FGATTN_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(mask) & 3u) return FGATTN_ERR_INVALID_ARG;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FGATTN_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 96 && d != 128) return FGATTN_ERR_UNSUPPORTED;
     if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
     if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;
     const int64_t cap = fgattn_kept_capacity(L);

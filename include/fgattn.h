@@ -98,7 +98,10 @@ fgattn_status fgattn_compact_mask(const uint32_t* mask, int64_t B, int64_t H, in
  *                  every count must be >= 1 and <= cap
  *   out       out  device bf16 [B][H][L][d]
  *   lse       out  device fp32 [B][H][L], may be NULL
- * Supported: d in {64, 128}, M in {16, 32, 64, 128}, any N >= 1, any L >= 1.
+ * Supported: d in {64, 96, 128}, M in {16, 32, 64, 128}, any N >= 1, any L >= 1.
+ * (At d = 96 the P.V product runs on V padded with zero columns to 128: the
+ * tensor-core shape of that product needs 64 or 128; the padding is never
+ * stored.)
  * Accumulation in fp32; P is rounded to bf16 for the P.V product; the sum l
  * is taken over the fp32 probabilities.
  * Errors: INVALID_ARG, UNSUPPORTED, CAPACITY, CUDA.  Kernel-side problems

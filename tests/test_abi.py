@@ -83,7 +83,7 @@ def _cmp(**kw):
     (dict(cap=63), F.ERR_CAPACITY),
     (dict(cap=66), F.ERR_CAPACITY),
     (dict(idx=P + 4), F.ERR_INVALID_ARG),
-    (dict(d=96), F.ERR_UNSUPPORTED),
+    (dict(d=80), F.ERR_UNSUPPORTED),
     (dict(d=256), F.ERR_UNSUPPORTED),
     (dict(M=48), F.ERR_UNSUPPORTED),
     (dict(M=8), F.ERR_UNSUPPORTED),
@@ -139,7 +139,7 @@ def test_header_declares_strided_forward():
     (dict(ks=(64 * 4 * 128, 136, 4 * 136)), F.ERR_INVALID_ARG),    # k strides not whole rows
     (dict(vs=(64 * 4 * 128, 128, 4 * 128 + 8)), F.ERR_INVALID_ARG),  # v token stride not whole rows
     (dict(os_=(64 * 4 * 128, 128, -512)), F.ERR_INVALID_ARG),      # negative stride
-    (dict(d=96), F.ERR_UNSUPPORTED),
+    (dict(d=80), F.ERR_UNSUPPORTED),
     (dict(cap=63), F.ERR_CAPACITY),
 ])
 def test_forward_strided_rejects(kw, status):
@@ -179,7 +179,7 @@ def _from_host(**kw):
     (dict(hpg=0), F.ERR_INVALID_ARG),
     (dict(idx=P + 4), F.ERR_INVALID_ARG),
     (dict(cap=60), F.ERR_CAPACITY),
-    (dict(d=96), F.ERR_UNSUPPORTED),
+    (dict(d=80), F.ERR_UNSUPPORTED),
     (dict(M=48), F.ERR_UNSUPPORTED),
 ])
 def test_from_host_rejects(kw, status):

@@ -53,6 +53,10 @@ FUZZ = [
     # keys of a chunk split unevenly between the two softmax halves
     (100, 128, 128, 16, 0.5, 1), (1, 128, 128, 1, 1.0, 1), (256, 64, 128, 128, 0.3, 2), (384, 128, 128, 32, 0.2, 1),
     (200, 128, 128, 5, 0.35, 1),
+    # d = 96 (Q/K second panel of 32 columns, V and O padded to 128): every kernel and layout
+    (300, 96, 64, 16, 0.3, 2), (257, 96, 64, 1, 0.4, 1), (200, 96, 16, 3, 0.5, 1), (640, 96, 32, 64, 0.5, 1),
+    (130, 96, 32, 4, 0.3, 1), (513, 96, 128, 3, 0.3, 1), (384, 96, 128, 32, 0.2, 1), (97, 96, 128, 128, 1.0, 1),
+    (700, 96, 64, 7, 0.1, 1),
 ]
 
 
@@ -82,12 +86,12 @@ def test_large_scores_rescale(oracle):
     parity_case(oracle, q, k, v, W.pack_tiles(tiles), M, N, 0.3)
 
 
-@pytest.mark.parametrize("M", [64, 128])
-def test_dense_null_list_matches_all_ones(oracle, M):
+@pytest.mark.parametrize("M,d", [(64, 128), (128, 128), (64, 96), (128, 96)])
+def test_dense_null_list_matches_all_ones(oracle, M, d):
     """A dense run (no lists) equals an all-ones mask.  Dense runs and M = 128 lists take
     the query-major kernel (identical values); M = 64 lists take the key-major one
     (same result within tolerance, both checked against the oracle)."""
-    L, d, N = 777, 128, 16
+    L, N = 777, 16
     QB, G = -(-L // M), -(-L // N)
     q, k, v = W.random_qkv(2, 2, L, d, seed=8)
     ones = W.pack_tiles(np.ones((2, 2, QB, G), bool))
@@ -113,13 +117,15 @@ def _inputs(name, N, sp):
 # call).  Each is checked against the oracle on the first block, the ragged last
 # blocks, at least 256 further seeded blocks and one whole head; the per-key
 # layer (1024 blocks) on every block.  The oracle's cost grows with the kept
-# scores, so the densest HunyuanVideo-like point (0 %) takes its whole-launch
-# check from the dense run of the same kernel instead (below).
+# scores, so on the HunyuanVideo-like layer (929 blocks of 128 rows x 118800
+# keys per head) the whole head is checked at 70 % and 90 %, and the densest
+# point (0 %) takes its whole-launch check from the dense run of the same
+# kernel instead (below).
 @pytest.mark.parametrize("name,N,sp,whole_head", [
     ("perkey", None, None, None),
     ("wan480p", None, None, 0),
     ("hunyuan720p", None, 0.0, None),
-    ("hunyuan720p", None, 0.5, 0),
+    ("hunyuan720p", None, 0.5, None),
     ("hunyuan720p", None, 0.7, 0),
     ("hunyuan720p", None, 0.9, 0),
     ("gransweep", 1, None, 0),
@@ -143,6 +149,18 @@ def test_workload_sampled_blocks(oracle, name, N, sp, whole_head):
         o2, l2, _, _ = run_gpu(q, k, v, mask, w.M, N, w.scale, dense=True)
         assert torch.equal(out, o2) and torch.equal(lse, l2)
     print(name, N, sp, stats)
+
+
+def test_head_dim_96_wan_like_layer(oracle):
+    """d = 96 at the Wan-480p-like shape and mask (4 heads): 256 seeded blocks, the ragged
+    last blocks and one whole head against the oracle."""
+    w = W.get("wan480p").with_(H=4, d=96)
+    q, k, v = W.make_qkv(w, 0)
+    mask = W.make_mask(w, 0)
+    blocks = sample_blocks(w.B, w.H, w.QB, 256, seed=13, whole_heads=(1,))
+    stats, (out, lse, _, _) = parity_case(oracle, q, k, v, mask, w.M, w.N, w.scale, blocks=blocks)
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    print(stats)
 
 
 @pytest.mark.parametrize("M", [64, 128])

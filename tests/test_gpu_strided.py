@@ -19,6 +19,9 @@ CASES = [
     (2, 2, 300, 64, 32, 8, 0.4, False),     # d = 64
     (1, 2, 650, 128, 128, 64, 0.5, False),  # M = 128
     (2, 2, 400, 128, 64, 16, 1.0, True),    # dense run (no lists)
+    (2, 2, 333, 96, 64, 16, 0.4, False),    # d = 96, tile layout
+    (1, 3, 290, 96, 32, 5, 0.3, False),     # d = 96, gather layout
+    (1, 2, 300, 96, 128, 16, 0.5, False),   # d = 96, M = 128
 ]
 
 
