@@ -60,7 +60,10 @@ __device__ unsigned int g_device_error = 0u;
 constexpr uint32_t kErrBadIndex = 0x1u;
 constexpr uint32_t kErrBadCount = 0x2u;
 constexpr uint32_t kErrTimeout = 0x4u;
-constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
+#ifndef FGATTN_WAIT_TIMEOUT_NS
+#define FGATTN_WAIT_TIMEOUT_NS 2000000000ull  // 2 s per wait
+#endif
+constexpr unsigned long long kWaitTimeoutNs = FGATTN_WAIT_TIMEOUT_NS;
 
 // Layouts (template parameter STRIDED).  Contiguous: q, k, v, out are
 // [B][H][L][D]; the tile maps (q, k16, v16) and the gather map (k) are 2-D over
@@ -464,7 +467,7 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
         constexpr int DP = C::DP;
         constexpr int PPR = DP / 8;    // 16-byte pieces per row of a V slot (padding pieces zero-filled)
         constexpr int RPI = 32 / PPR;  // rows per warp instruction
-        int64_t g = 0;
+        int64_t g = 0, v_issued = 0;  // v_issued: chunks this warp has issued
         bool ok = true;
         for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
             const int64_t bh = item / p.QB;
@@ -546,10 +549,16 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                     }
                 }
                 ptx::cp_async_arrive_noinc(BAR(C::B_VFULL + st));
+                ++v_issued;
             }
             g += nch;
         }
         ptx::cp_async_wait_all();
+        // Every V box this warp issued has landed before the block exits: on the normal
+        // path the P.V issuer has consumed them all, after an abort nobody else waits
+        // for them (a block must not exit with bulk copies into its shared memory in flight).
+        for (int64_t i = v_issued > NV ? v_issued - NV : 0; i < v_issued; ++i)
+            bounded_wait(BAR(C::B_VFULL + (int)(i % NV)), (uint32_t)((i / NV) & 1), abort_flag, false);
     } else if (warp == AW + 3 || (!GATHER && warp == AW + 2)) {
         // ===================================================== MMA issuers
         // Two issuing threads, one per MMA kind, so that neither waits behind the

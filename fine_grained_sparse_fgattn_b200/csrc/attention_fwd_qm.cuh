@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
         constexpr int DP = C::DP;
         constexpr int PPR = DP / 8;     // 16-byte pieces per row of a V slot (padding pieces zero-filled)
         constexpr int RPI = 32 / PPR;   // rows per warp instruction
-        int64_t g = 0;
+        int64_t g = 0, v_issued = 0;  // v_issued: chunks this warp has issued
         bool ok = true;
         for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
             const int64_t bh = item / p.QB;
@@ -341,10 +341,16 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                     }
                 }
                 ptx::cp_async_arrive_noinc(BAR(C::B_VFULL + st));
+                ++v_issued;
             }
             g += nch;
         }
         ptx::cp_async_wait_all();
+        // Every V box this warp issued has landed before the block exits: on the normal
+        // path the P.V issuer has consumed them all, after an abort nobody else waits
+        // for them (a block must not exit with bulk copies into its shared memory in flight).
+        for (int64_t i = v_issued > NV ? v_issued - NV : 0; i < v_issued; ++i)
+            bounded_wait(BAR(C::B_VFULL + (int)(i % NV)), (uint32_t)((i / NV) & 1), abort_flag, false);
     } else if (warp == 8) {
         // ===================================================== MMA issuer
         ptx::regs_dec<C::AUX_REGS>();

@@ -90,11 +90,70 @@ int current_sms() {
     return sms;
 }
 
+// A tensor map is a pure function of a buffer's address, shape, strides and box, so
+// the map set of a launch is cached under everything that determines it; repeated
+// calls on the same buffers (the usual case for a layer called every denoising step)
+// skip the host-side encodes.  Sixteen sets, replaced round-robin.
+struct MapSetKey {
+    const void* q;
+    const void* k;
+    const void* v;
+    int64_t st[9];  // q, k, v strides
+    int64_t B, H, L, d, k_rows;
+    uint32_t mq;
+    bool strided;
+    bool operator==(const MapSetKey& o) const {
+        if (q != o.q || k != o.k || v != o.v || B != o.B || H != o.H || L != o.L || d != o.d || k_rows != o.k_rows ||
+            mq != o.mq || strided != o.strided)
+            return false;
+        for (int i = 0; i < 9; ++i)
+            if (st[i] != o.st[i]) return false;
+        return true;
+    }
+};
+struct MapSet {
+    CUtensorMap q, k, k16, v16, q_hi, k_hi, k16_hi;
+};
+constexpr int kMapCacheSize = 16;
+std::mutex g_map_mutex;
+MapSetKey g_map_keys[kMapCacheSize];
+MapSet g_map_sets[kMapCacheSize];
+bool g_map_valid[kMapCacheSize] = {};
+int g_map_next = 0;
+
+template <bool STRIDED>
+bool encode_maps_uncached(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
+                          const void* v, const Strides& vs, int64_t B, int64_t H, int64_t d, int64_t k_rows,
+                          uint32_t mq);
+
 // The tensor maps of one launch: query tiles of mq rows, k row gathers, 16-key k and v
 // boxes; at d = 96 also the 32-column maps of columns 64..95 of q and k.
 template <bool STRIDED>
 bool encode_maps(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
                  const void* v, const Strides& vs, int64_t B, int64_t H, int64_t d, int64_t k_rows, uint32_t mq) {
+    MapSetKey key = {q, k, v, {qs.s[0], qs.s[1], qs.s[2], ks.s[0], ks.s[1], ks.s[2], vs.s[0], vs.s[1], vs.s[2]},
+                     B, H, prm.L, d, k_rows, mq, STRIDED};
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    for (int i = 0; i < kMapCacheSize; ++i)
+        if (g_map_valid[i] && g_map_keys[i] == key) {
+            const MapSet& m = g_map_sets[i];
+            prm.tmap_q = m.q, prm.tmap_k = m.k, prm.tmap_k16 = m.k16, prm.tmap_v16 = m.v16;
+            prm.tmap_q_hi = m.q_hi, prm.tmap_k_hi = m.k_hi, prm.tmap_k16_hi = m.k16_hi;
+            return true;
+        }
+    if (!encode_maps_uncached<STRIDED>(prm, q, qs, k, ks, v, vs, B, H, d, k_rows, mq)) return false;
+    const int i = g_map_next;
+    g_map_next = (g_map_next + 1) % kMapCacheSize;
+    g_map_keys[i] = key;
+    g_map_sets[i] = {prm.tmap_q, prm.tmap_k, prm.tmap_k16, prm.tmap_v16, prm.tmap_q_hi, prm.tmap_k_hi, prm.tmap_k16_hi};
+    g_map_valid[i] = true;
+    return true;
+}
+
+template <bool STRIDED>
+bool encode_maps_uncached(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
+                          const void* v, const Strides& vs, int64_t B, int64_t H, int64_t d, int64_t k_rows,
+                          uint32_t mq) {
     const int64_t L = prm.L;
     const bool narrow = d == 96;
     if (STRIDED) {
@@ -342,6 +401,7 @@ fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* b
 }
 
 int fgattn_num_sms(void) { return current_sms(); }
+
 
 const char* fgattn_status_string(fgattn_status status) {
     switch (status) {

@@ -143,9 +143,13 @@ __global__ void __launch_bounds__(128, 1) probe_rows_kernel(const __grid_constan
 }
 
 // tcgen05.mma issue rate.  which = 1: score products only; 2: P.V products only;
-// 3: both, alternating per chunk as in the key-major kernel.  One thread issues
-// `chunks` groups of 8 MMAs per kind, committing each group to a barrier, and
-// waits for the commit of the group two back (the kernels' double buffering).
+// 3: both, one group of 8 after the other per chunk; 4: both, interleaved MMA by
+// MMA (score k-step i, then P.V k-step i); 5: score products with the 8 k-steps
+// alternating between two accumulators (two independent chains).  One thread
+// issues `chunks` groups of 8 MMAs per kind, committing each group to a barrier,
+// and waits for the commit of the group two back (the kernels' double buffering).
+// Modes 4 and 5 separate the tensor pipe's throughput from the latency of a chain
+// of dependent accumulations into one accumulator.
 template <int N>
 __global__ void __launch_bounds__(128, 1) probe_mma_kernel(int which, uint32_t chunks, unsigned long long* cycles) {
     constexpr int D = 128;
@@ -192,7 +196,34 @@ __global__ void __launch_bounds__(128, 1) probe_mma_kernel(int which, uint32_t c
         const uint64_t t0 = clock64();
         bool ok = true;
         uint32_t n1 = 0, n2 = 0;  // commits per kind
-        for (uint32_t c = 0; c < chunks && ok; ++c) {
+        for (uint32_t c = 0; c < chunks && ok && which == 4; ++c) {
+            if (n1 >= 2) ok = ok && wait_bounded(sbase + OFF_BAR + 8u * (n1 & 1), ((n1 - 2) >> 1) & 1u);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t koff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
+                const uint32_t qoff = (uint32_t)(kk / 4) * (N * 128) + (uint32_t)(kk % 4) * 32u;
+                ptx::mma_bf16_ss(tS, umma_desc_join(klo + (koff >> 4), HI_KQ), umma_desc_join(qlo + (qoff >> 4), HI_KQ),
+                                 IDESC1, kk > 0 ? 1u : 0u);
+                ptx::mma_bf16_ss(tO, umma_desc_join(vlo + (uint32_t)(kk * 2048 >> 4), HI_V),
+                                 umma_desc_join(plo + (uint32_t)(kk * 16 * P_ROW >> 4), HI_P), IDESC2,
+                                 (c > 0 || kk > 0) ? 1u : 0u);
+            }
+            ptx::mma_commit(sbase + OFF_BAR + 8u * (n1 & 1));
+            ++n1;
+        }
+        for (uint32_t c = 0; c < chunks && ok && which == 5; ++c) {
+            if (n1 >= 2) ok = ok && wait_bounded(sbase + OFF_BAR + 8u * (n1 & 1), ((n1 - 2) >> 1) & 1u);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t koff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
+                const uint32_t qoff = (uint32_t)(kk / 4) * (N * 128) + (uint32_t)(kk % 4) * 32u;
+                ptx::mma_bf16_ss(kk & 1 ? tO : tS, umma_desc_join(klo + (koff >> 4), HI_KQ),
+                                 umma_desc_join(qlo + (qoff >> 4), HI_KQ), IDESC1, kk > 1 ? 1u : 0u);
+            }
+            ptx::mma_commit(sbase + OFF_BAR + 8u * (n1 & 1));
+            ++n1;
+        }
+        for (uint32_t c = 0; c < chunks && ok && which <= 3; ++c) {
             if (which & 1) {
                 if (n1 >= 2) ok = ok && wait_bounded(sbase + OFF_BAR + 8u * (n1 & 1), ((n1 - 2) >> 1) & 1u);
 #pragma unroll
@@ -345,7 +376,7 @@ int fgprobe_rows(int mode, const void* src, int64_t rows, int chunks, int reps, 
 // SM clocks block 0 spent from the first issue to the last completion.
 int fgprobe_mma(int which, int n, int chunks, int reps, void* stream, float* ms, double* flops,
                 unsigned long long* cycles_dev, unsigned long long* cycles) {
-    if (which < 1 || which > 3 || chunks < 1 || reps < 1 || !ms || !flops || !cycles_dev || !cycles) return 1;
+    if (which < 1 || which > 5 || chunks < 1 || reps < 1 || !ms || !flops || !cycles_dev || !cycles) return 1;
     if (n != 64 && n != 128 && n != 256) return 1;
     if (!clear_error()) return 4;
     const int grid = sms();
@@ -361,7 +392,8 @@ int fgprobe_mma(int which, int n, int chunks, int reps, void* stream, float* ms,
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 4;
     const int st = timed([&] { k<<<grid, 128, smem, s>>>(which, (uint32_t)chunks, cycles_dev); }, reps, s, ms);
     const double per_kind = 2.0 * 128.0 * n * 128.0;  // one chunk: M 128 x N x K 128
-    *flops = (double)grid * chunks * per_kind * ((which & 1) + ((which >> 1) & 1));
+    const int kinds = which == 3 || which == 4 ? 2 : 1;
+    *flops = (double)grid * chunks * per_kind * kinds;
     if (cudaMemcpy(cycles, cycles_dev, sizeof(unsigned long long), cudaMemcpyDeviceToHost) != cudaSuccess) return 4;
     return st ? st : probe_error();
 }

@@ -10,8 +10,11 @@ the attention path never loads) and prints one JSON object:
          16.8 MB, L2-resident) and of the whole layer (40 heads, 671 MB, from HBM).
   mma    tcgen05.mma kind::f16 with the key-major kernel's operand layouts,
          M = 128 and N in {64, 128, 256}: the score product alone, the P.V
-         product alone and both alternating, one commit per 8-MMA chunk.
-         Reported as TFLOP/s over the whole GPU and SM clocks per MMA.
+         product alone, both one group after the other, both interleaved MMA by
+         MMA, and the score product split over two accumulators; one commit per
+         8-MMA chunk.  Reported as TFLOP/s over the whole GPU and SM clocks per
+         MMA.  The last two separate the tensor pipe's throughput from the
+         latency of a chain of dependent accumulations.
   ex2    MUFU ex2 results per SM clock per SM.
 
   python -m fine_grained_sparse_fgattn_b200.probes [--out FILE]
@@ -67,13 +70,14 @@ def mma_rates(lib, chunks: int = 2048, reps: int = 5) -> dict:
     dev = torch.zeros(1, dtype=torch.int64, device="cuda")
     res = {}
     for n in (64, 128, 256):
-        for which, name in ((1, "scores"), (2, "pv"), (3, "both")):
+        for which, name in ((1, "scores"), (2, "pv"), (3, "both"), (4, "both_interleaved"),
+                            (5, "scores_two_accumulators")):
             ms, fl, cyc = ctypes.c_float(), ctypes.c_double(), ctypes.c_ulonglong()
             st = lib.fgprobe_mma(which, n, chunks, reps, _stream(), ctypes.byref(ms), ctypes.byref(fl),
                                  ctypes.c_void_p(dev.data_ptr()), ctypes.byref(cyc))
             if st != 0:
                 raise RuntimeError(f"fgprobe_mma({name}, N={n}) failed with status {st}")
-            mmas = chunks * 8 * (2 if which == 3 else 1)
+            mmas = chunks * 8 * (2 if which in (3, 4) else 1)
             res[f"N{n}_{name}"] = {"tflops": fl.value / (ms.value * 1e-3) / 1e12, "ms": ms.value,
                                    "clocks_per_mma": cyc.value / mmas,
                                    "ideal_clocks_per_mma": 2.0 * 128 * n * 16 / 8192.0}
