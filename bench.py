@@ -242,14 +242,16 @@ def cfg_dict(w, args, flush):
     return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "grid": list(w.grid), "d": w.d, "M": w.M, "N": w.N,
             "sparsity_target": w.sparsity, "mask": w.mask, "qkv": w.qkv, "seed": args.seed,
             "l2": l2, "parallelism": f"heads x{args.gpus} (weak)",
-            "path": "dense (no kept lists)" if getattr(args, "dense", False) else "tile-sparse (compaction + forward)",
+            "path": "dense (no kept lists)" if getattr(args, "dense", False) else
+            "tile-sparse, fused (the forward reads the mask; no kept lists)" if getattr(args, "fused", False) else
+            "tile-sparse (compaction + forward)",
             "layout": "[B][L][H][d]" if getattr(args, "layout", "bhld") == "blhd" else "[B][H][L][d]"}
 
 
 def profile_key(w, args):
     """Name of the committed ncu summary for this exact workload (None when overridden)."""
     if args.N is not None or args.sparsity is not None or args.heads is not None or args.dense or \
-            args.layout != "bhld":
+            args.layout != "bhld" or args.fused:
         return None
     return w.name
 
@@ -275,6 +277,9 @@ def main():
                          "[B][L][H][d] (strided entry point)")
     ap.add_argument("--dense", action="store_true",
                     help="dense run of the same kernel (no kept lists: every key of every block)")
+    ap.add_argument("--fused", action="store_true",
+                    help="one kernel per step: the forward reads the mask in place of kept lists "
+                         "(fgattn_masked_forward; compaction fused into the forward)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.get(args.workload)
@@ -311,12 +316,14 @@ def main():
     stream = torch.cuda.current_stream()
 
     def compact():
-        if not args.dense:
+        if not args.dense and not args.fused:
             F.compact_mask(mask, B, H, L, M, N, kept_idx=kept_idx, kept_cnt=kept_cnt, cap=cap)
 
     def forward():
         if args.dense:
             F.forward(q, k, v, None, None, M, N, w.scale, out=out, lse=lse)
+        elif args.fused:
+            F.masked_forward(q, k, v, mask, M, N, w.scale, out=out, lse=lse)
         else:
             F.forward(q, k, v, kept_idx, kept_cnt, M, N, w.scale, out=out, lse=lse)
 
@@ -324,6 +331,8 @@ def main():
         compact()
         forward()
 
+    if args.fused:  # the kept-key counts for the FLOP figure, once, outside any timing
+        F.compact_mask(mask, B, H, L, M, N, kept_idx=kept_idx, kept_cnt=kept_cnt, cap=cap)
     step()
     assert F.device_error() == 0, "device error on the first step"
     if args.dense:
@@ -392,7 +401,7 @@ def main():
     # Contiguous tile-sparse runs go through the host-to-host entry point, which overlaps
     # the copies of one head group with the kernels of another; dense and strided runs
     # copy in, run and copy out one after the other.
-    pipelined = args.layout == "bhld" and not args.dense
+    pipelined = args.layout == "bhld" and not args.dense and not args.fused
     buffers = {"q": q, "k": k, "v": v, "mask": mask, "kept_idx": kept_idx, "kept_cnt": kept_cnt, "out": out,
                "lse": lse}
 
@@ -428,13 +437,14 @@ def main():
     from fine_grained_sparse_fgattn_b200 import _build
     # 128-row query blocks (M = 128 lists, dense runs) run the query-major kernel
     qm = args.dense or M == 128
-    gather = not args.dense and N % 16 != 0
+    gather = not args.dense and min(N, L) % 16 != 0
     strided = args.layout != "bhld"
+    tf = lambda x: str(bool(x)).lower()
     if qm:
-        kname = f"fgattn_fwd_qm_kernel<{d},{str(gather).lower()},{str(strided).lower()}>"
+        kname = f"fgattn_fwd_qm_kernel<{d},{tf(gather)},{tf(strided)},{tf(args.fused)}>"
         traffic, _ = ncu_traffic(profile_key(w, args), _build.kernel_hash("fwd_qm"), "fgattn_fwd_qm")
     else:
-        kname = f"fgattn_fwd_kernel<{d},{M},{str(gather).lower()},{str(strided).lower()}>"
+        kname = f"fgattn_fwd_kernel<{d},{M},{tf(gather)},{tf(strided)},{tf(args.fused)}>"
         traffic, _ = ncu_traffic(profile_key(w, args), _build.kernel_hash("fwd"))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
@@ -463,7 +473,7 @@ def main():
                     "mode": (f"fgattn_attention_from_host: copies overlapped with the kernels, "
                              f"{args.heads_per_group} heads per group") if pipelined
                     else "copy in, run, copy out (serial)"},
-            "gpu_launches": (1 if args.dense else 2) * args.steps, "clocks": clocks,
+            "gpu_launches": (1 if args.dense or args.fused else 2) * args.steps, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -22,12 +22,14 @@ import torch
 
 from . import _build
 
-__all__ = ["kept_capacity", "compact_mask", "forward", "masked_forward_noalloc", "attention_from_host", "device_error", "status_string", "num_sms",
+__all__ = ["kept_capacity", "compact_mask", "forward", "masked_forward", "masked_forward_noalloc", "attention_from_host",
+           "device_error", "status_string", "num_sms", "FUSED_MAX_WORDS",
            "FgattnError", "LIB_PATH", "DEVERR_BAD_INDEX", "DEVERR_BAD_COUNT", "DEVERR_TIMEOUT"]
 
 LIB_PATH = _build.LIB
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_DEVICE = range(6)
+FUSED_MAX_WORDS = 256  # mask words per query block that fgattn_masked_forward reads in place
 DEVERR_BAD_INDEX, DEVERR_BAD_COUNT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 
@@ -51,6 +53,8 @@ def _load() -> ctypes.CDLL:
     lib.fgattn_attention_from_host.argtypes = [p, p, p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64,
                                                ctypes.c_float, p, p, p, p, i64, p]
     lib.fgattn_attention_from_host.restype = i32
+    lib.fgattn_masked_forward.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64, ctypes.c_float, p, p, p]
+    lib.fgattn_masked_forward.restype = i32
     lib.fgattn_masked_forward_noalloc.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64, ctypes.c_float, p, p, p]
     lib.fgattn_masked_forward_noalloc.restype = i32
     lib.fgattn_device_error.argtypes = [p, i32, ctypes.POINTER(ctypes.c_uint32)]
@@ -295,6 +299,36 @@ def attention_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask:
         _dev(b["out"], "out buffer", bf), _dev(b["lse"], "lse buffer", (torch.float32,)),
         _host(out, "out", bf), _host(lse, "lse", (torch.float32,)), int(heads_per_group), _stream_ptr(stream))
     _check(st, "fgattn_attention_from_host")
+    return out, lse
+
+
+def masked_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: torch.Tensor, M: int, N: int,
+                   scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                   lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Mask -> (out, lse) in one kernel: the forward reads the packed tile mask in place of
+    kept lists (each warp expands its query block's row itself), so no list is written or
+    read and nothing is allocated beyond out and lse.  q, k, v: contiguous bf16 [B,H,L,d];
+    mask: int32/uint32 [B,H,QB,W] with W <= FUSED_MAX_WORDS (else FgattnError UNSUPPORTED:
+    use compact_mask + forward).  Results equal compact_mask + forward bit for bit."""
+    B, H, L, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, H, L, d] shape")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if min(L, M, N) >= 1:
+        QB, W = _geometry(L, M, N)
+        _numel(mask, B * H * QB * W, "mask")
+    if out is None:
+        out = torch.empty_like(q)
+    if out.shape != q.shape:
+        raise ValueError("out must have the shape of q")
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _numel(lse, B * H * L, "lse")
+    bf = (torch.bfloat16,)
+    st = _lib.fgattn_masked_forward(_dev(q, "q", bf), _dev(k, "k", bf), _dev(v, "v", bf),
+                                    _dev(mask, "mask", (torch.int32, torch.uint32)), B, H, L, d, M, N, scale,
+                                    _dev(out, "out", bf), _dev(lse, "lse", (torch.float32,)), _stream_ptr(stream))
+    _check(st, "fgattn_masked_forward")
     return out, lse
 
 

@@ -51,6 +51,7 @@
 
 #include <cstdint>
 
+#include "mask_row.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fgattn {
@@ -89,8 +90,11 @@ struct alignas(64) FwdParams {
     int32_t k_ul, v_ul;  // k / v token strides in rows of D elements
     int64_t o_sb, o_sh, o_sl;  // out element strides
     int64_t H;
-    const int32_t* kept_idx;  // nullptr: dense (every key kept)
+    const int32_t* kept_idx;  // nullptr: dense (every key kept), or the mask below
     const int32_t* kept_cnt;
+    // fused kernels only: the packed tile mask, read instead of kept lists
+    const uint32_t* mask;
+    int64_t mask_w, mask_g, mask_n;  // words per row, key groups, keys per group
     __nv_bfloat16* out;
     float* lse;  // may be nullptr
     int64_t cap;
@@ -266,6 +270,31 @@ __device__ __forceinline__ int4 fetch_idx(const int32_t* lst, int64_t cnt, int64
                      j0 + 2 < cnt ? __ldg(lst + j0 + 2) : 0, j0 + 3 < cnt ? __ldg(lst + j0 + 3) : 0);
 }
 
+// Fused kernels: list entries 4*lane .. 4*lane+3 of chunk c from the mask row
+// (warp-collective; every lane of the warp calls it).
+__device__ __forceinline__ int4 fused_idx4(const MaskRow& mr, int64_t n, int64_t c, int lane4, int lane) {
+    const int64_t j0 = c * 128 + 4 * lane4;
+    if (n % 4 == 0) {  // four consecutive keys of one group
+        const int32_t k = mask_row_key(mr, j0, n, lane);
+        return make_int4(j0 < mr.keys ? k : 0, j0 + 1 < mr.keys ? k + 1 : 0, j0 + 2 < mr.keys ? k + 2 : 0,
+                         j0 + 3 < mr.keys ? k + 3 : 0);
+    }
+    return make_int4(mask_row_key(mr, j0, n, lane), mask_row_key(mr, j0 + 1, n, lane),
+                     mask_row_key(mr, j0 + 2, n, lane), mask_row_key(mr, j0 + 3, n, lane));
+}
+
+// Kept keys of work item `item`: from kept_cnt, L for a dense run, or the mask
+// row (fused kernels; warp-collective, and `mr` keeps the row for the caller).
+template <bool FUSED, int MQ>
+__device__ __forceinline__ int64_t item_keys(const FwdParams& p, int64_t item, bool report, MaskRow& mr, int lane) {
+    if constexpr (FUSED) {
+        mask_row_load(mr, p.mask, item, p.QB, MQ, p.mask_n, p.mask_g, p.mask_w, p.L, lane);
+        return mr.keys;
+    } else {
+        return item_count(p, item, report);
+    }
+}
+
 // Gather-map row coordinates of four fetched entries: row0 + key * stride.
 // Entries outside [0, L) are reported and replaced by key 0 of the head (as are
 // entries past the list, whose scores the softmax masks).
@@ -286,7 +315,7 @@ __device__ __forceinline__ void rows_of(const FwdParams& p, int4 raw, int64_t ro
     }
 }
 
-template <int D, int MQ, bool GATHER, bool STRIDED>
+template <int D, int MQ, bool GATHER, bool STRIDED, bool FUSED>
 __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
     fgattn_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = FwdCfg<D, MQ, GATHER>;
@@ -372,9 +401,18 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                 hi = (int32_t)(bh - (int64_t)bi * p.H);
                 krow0 = bi * p.k_ub + hi * p.k_uh;
             }
-            const int64_t cnt = item_count(p, item, kw == 0 && lane == 0);
+            MaskRow mr;
+            const int64_t cnt = item_keys<FUSED, MQ>(p, item, kw == 0 && lane == 0, mr, lane);
             const int64_t nch = (cnt + 127) / 128;
             const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
+            auto fetch4 = [&](int64_t c) -> int4 {  // this lane's four entries of chunk c (-1: none)
+                if constexpr (FUSED) {
+                    const int4 e = fused_idx4(mr, p.mask_n, c, g4, lane);  // every lane takes part
+                    return issuer ? e : make_int4(-1, -1, -1, -1);
+                } else {
+                    return issuer ? fetch_idx(lst, cnt, c, g4) : make_int4(-1, -1, -1, -1);
+                }
+            };
             if (kw == 0) {  // the query tile (rows past L are padding; their results are never stored)
                 const bool okq = it == 0 || bounded_wait(BAR(C::B_QEMPTY), (uint32_t)((it - 1) & 1), abort_flag);
                 if (!__all_sync(0xffffffffu, okq)) {
@@ -400,15 +438,14 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
             constexpr int PF = 4;  // index prefetch distance in chunks (the lists live in HBM)
             int4 ring[PF];
 #pragma unroll
-            for (int i = 0; i < PF; ++i)
-                ring[i] = (issuer && i < nch) ? fetch_idx(lst, cnt, i, g4) : make_int4(-1, -1, -1, -1);
+            for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch4(i) : make_int4(-1, -1, -1, -1);
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
                 const int st = (int)(gc % NK);
                 const int4 cur = ring[0];
 #pragma unroll
                 for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
-                ring[PF - 1] = (issuer && c + PF < nch) ? fetch_idx(lst, cnt, c + PF, g4) : make_int4(-1, -1, -1, -1);
+                ring[PF - 1] = c + PF < nch ? fetch4(c + PF) : make_int4(-1, -1, -1, -1);
                 const bool okw =
                     gc < NK || bounded_wait(BAR(C::B_KEMPTY + st), (uint32_t)((gc / NK - 1) & 1), abort_flag);
                 if (!__all_sync(0xffffffffu, okw)) {
@@ -471,7 +508,8 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
         bool ok = true;
         for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
             const int64_t bh = item / p.QB;
-            const int64_t cnt = item_count(p, item, false);
+            MaskRow mr;
+            const int64_t cnt = item_keys<FUSED, MQ>(p, item, false, mr, lane);
             const int64_t nch = (cnt + 127) / 128;
             const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
             const __nv_bfloat16* vb = p.v_base + (size_t)bh * L * D;
@@ -483,8 +521,13 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
             }
             auto fetch1 = [&](int64_t c) -> int32_t {
                 const int64_t j = c * 128 + vw * 32 + lane;
-                if (j >= cnt) return -1;  // past the list
-                return lst ? __ldg(lst + j) : (int32_t)j;
+                if constexpr (FUSED) {
+                    const int32_t k = mask_row_key(mr, j, p.mask_n, lane);  // every lane takes part
+                    return j >= cnt ? -1 : k;
+                } else {
+                    if (j >= cnt) return -1;  // past the list
+                    return lst ? __ldg(lst + j) : (int32_t)j;
+                }
             };
             constexpr int PF = 4;
             int32_t ring[PF];
@@ -567,7 +610,7 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
         // soon as its V rows and probabilities are ready.  The tensor pipe takes the
         // two streams in arrival order; each thread's commits track its own MMAs.
         if constexpr (C::AUX_REGS != C::LAUNCH_REGS) ptx::regs_dec<C::AUX_REGS>();
-        if (lane == 0) {
+        {
             constexpr uint32_t IDESC1 = umma_idesc_bf16(128, MQ, false, false);
             constexpr uint32_t IDESC2 = umma_idesc_bf16(C::DP, MQ, true, true);
             constexpr uint32_t P_LAYOUT = (C::P_ROW == 128) ? 2u : (C::P_ROW == 64) ? 4u : 6u;
@@ -620,27 +663,35 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
                 ptx::mma_commit(BAR(C::B_SFULL + s));
                 return true;
             };
+            // The whole warp walks the items (a fused kernel reads each item's mask row
+            // with all lanes); lane 0 issues and commits.
             int64_t g = 0, it = 0;
             for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
-                const int64_t nch = (item_count(p, item, false) + 127) / 128;
-                if constexpr (GATHER) {
-                    // one issuing thread: S of chunks 0 and 1, then for every chunk c the
-                    // S of chunk c+2 (its slot frees early in softmax(c)) before the P.V of c
-                    for (int64_t c = 0; c < nch && c < 2 && ok; ++c) ok = issue_s(g + c, c, it);
-                    for (int64_t c = 0; c < nch && ok; ++c) {
-                        if (c + 2 < nch) ok = issue_s(g + c + 2, c + 2, it);
-                        if (ok) ok = issue_pv(g + c, c);
+                MaskRow mr;
+                const int64_t nch = (item_keys<FUSED, MQ>(p, item, false, mr, lane) + 127) / 128;
+                if (lane == 0) {
+                    if constexpr (GATHER) {
+                        // one issuing thread: S of chunks 0 and 1, then for every chunk c the
+                        // S of chunk c+2 (its slot frees early in softmax(c)) before the P.V of c
+                        for (int64_t c = 0; c < nch && c < 2 && ok; ++c) ok = issue_s(g + c, c, it);
+                        for (int64_t c = 0; c < nch && ok; ++c) {
+                            if (c + 2 < nch) ok = issue_s(g + c + 2, c + 2, it);
+                            if (ok) ok = issue_pv(g + c, c);
+                        }
+                    } else {
+                        for (int64_t c = 0; c < nch && ok; ++c)
+                            ok = (warp == AW + 3) ? issue_s(g + c, c, it) : issue_pv(g + c, c);
                     }
-                } else {
-                    for (int64_t c = 0; c < nch && ok; ++c)
-                        ok = (warp == AW + 3) ? issue_s(g + c, c, it) : issue_pv(g + c, c);
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
                 g += nch;
             }
             // drain: every MMA this thread issued has completed before TMEM is freed
-            const int drain = (warp == AW + 3) ? C::B_DRAIN : C::B_DRAIN2;
-            ptx::mma_commit(BAR(drain));
-            bounded_wait(BAR(drain), 0u, abort_flag, /*honour_abort=*/false);
+            if (lane == 0) {
+                const int drain = (warp == AW + 3) ? C::B_DRAIN : C::B_DRAIN2;
+                ptx::mma_commit(BAR(drain));
+                bounded_wait(BAR(drain), 0u, abort_flag, /*honour_abort=*/false);
+            }
         }
         __syncwarp();
     } else {
@@ -665,7 +716,11 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
         for (int64_t item = blockIdx.x; item < p.items; item += gridDim.x) {
             const int64_t bh = item / p.QB;
             const int64_t qb = item - bh * p.QB;
-            const int64_t cnt = item_count(p, item, false);
+            int64_t cnt;
+            {
+                MaskRow mr;
+                cnt = item_keys<FUSED, MQ>(p, item, false, mr, lane);
+            }
             const int64_t nch = (cnt + 127) / 128;
             if (t < CW) mref[t] = -INFINITY;
             float lp[CW];

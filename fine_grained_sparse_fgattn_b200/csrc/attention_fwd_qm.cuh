@@ -84,7 +84,7 @@ struct QmCfg {
     static_assert(256 * SOFT_REGS + 256 * AUX_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
-template <int D, bool GATHER, bool STRIDED>
+template <int D, bool GATHER, bool STRIDED, bool FUSED>
 __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_constant__ FwdParams p) {
     using C = QmCfg<D, GATHER>;
     constexpr int NK = C::NK, NV = C::NV, MQ = C::MQ;
@@ -161,9 +161,18 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                     hi = (int32_t)(bh - (int64_t)bi * p.H);
                     krow0 = bi * p.k_ub + hi * p.k_uh;
                 }
-                const int64_t cnt = item_count(p, item, kw == 0 && lane == 0);
+                MaskRow mr;
+                const int64_t cnt = item_keys<FUSED, MQ>(p, item, kw == 0 && lane == 0, mr, lane);
                 const int64_t nch = (cnt + 127) / 128;
                 const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
+                auto fetch4 = [&](int64_t c) -> int4 {  // this lane's four entries of chunk c (-1: none)
+                    if constexpr (FUSED) {
+                        const int4 e = fused_idx4(mr, p.mask_n, c, g4, lane);  // every lane takes part
+                        return issuer ? e : make_int4(-1, -1, -1, -1);
+                    } else {
+                        return issuer ? fetch_idx(lst, cnt, c, g4) : make_int4(-1, -1, -1, -1);
+                    }
+                };
                 if (kw == 0) {  // the query tile (rows past L are padding; never stored)
                     const bool okq =
                         it == 0 || bounded_wait(BAR(C::B_QEMPTY), (uint32_t)((it - 1) & 1), abort_flag);
@@ -190,16 +199,14 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                 constexpr int PF = 4;  // index prefetch distance in chunks (the lists live in HBM)
                 int4 ring[PF];
 #pragma unroll
-                for (int i = 0; i < PF; ++i)
-                    ring[i] = (issuer && i < nch) ? fetch_idx(lst, cnt, i, g4) : make_int4(-1, -1, -1, -1);
+                for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch4(i) : make_int4(-1, -1, -1, -1);
                 for (int64_t c = 0; c < nch; ++c) {
                     const int64_t gc = g + c;
                     const int st = (int)(gc % NK);
                     const int4 cur = ring[0];
 #pragma unroll
                     for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
-                    ring[PF - 1] =
-                        (issuer && c + PF < nch) ? fetch_idx(lst, cnt, c + PF, g4) : make_int4(-1, -1, -1, -1);
+                    ring[PF - 1] = c + PF < nch ? fetch4(c + PF) : make_int4(-1, -1, -1, -1);
                     const bool okw =
                         gc < NK || bounded_wait(BAR(C::B_KEMPTY + st), (uint32_t)((gc / NK - 1) & 1), abort_flag);
                     if (!__all_sync(0xffffffffu, okw)) {
@@ -263,7 +270,8 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
         bool ok = true;
         for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
             const int64_t bh = item / p.QB;
-            const int64_t cnt = item_count(p, item, false);
+            MaskRow mr;
+            const int64_t cnt = item_keys<FUSED, MQ>(p, item, false, mr, lane);
             const int64_t nch = (cnt + 127) / 128;
             const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
             const __nv_bfloat16* vb = p.v_base + (size_t)bh * L * D;
@@ -275,8 +283,13 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
             }
             auto fetch1 = [&](int64_t c) -> int32_t {
                 const int64_t j = c * 128 + vw * 32 + lane;
-                if (j >= cnt) return -1;  // past the list
-                return lst ? __ldg(lst + j) : (int32_t)j;
+                if constexpr (FUSED) {
+                    const int32_t k = mask_row_key(mr, j, p.mask_n, lane);  // every lane takes part
+                    return j >= cnt ? -1 : k;
+                } else {
+                    if (j >= cnt) return -1;  // past the list
+                    return lst ? __ldg(lst + j) : (int32_t)j;
+                }
             };
             constexpr int PF = 4;
             int32_t ring[PF];
@@ -354,7 +367,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
     } else if (warp == 8) {
         // ===================================================== MMA issuer
         ptx::regs_dec<C::AUX_REGS>();
-        if (lane == 0) {
+        {
             constexpr uint32_t IDESC1 = umma_idesc_bf16(128, 128, false, false);  // S = Q . K^T
             constexpr uint32_t IDESC2 = umma_idesc_bf16(128, C::DP, false, true);  // O += P . V, V N-major
             constexpr uint32_t HI_V = umma_desc_hi(1024u, 2u);   // V rows: N-major, 128B swizzle
@@ -400,21 +413,29 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                 ptx::mma_commit(BAR(C::B_ODONE + (int)(gc & 1)));
                 return true;
             };
+            // The whole warp walks the items (a fused kernel reads each item's mask row
+            // with all lanes); lane 0 issues and commits.
             int64_t g = 0, it = 0;
             for (int64_t item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
-                const int64_t nch = (item_count(p, item, false) + 127) / 128;
-                // S of chunks 0 and 1, then for every chunk c the S of chunk c+2 (its slot
-                // frees as soon as the softmax has read chunk c) before the P.V of chunk c
-                for (int64_t c = 0; c < nch && c < 2 && ok; ++c) ok = issue_s(g + c, c, it);
-                for (int64_t c = 0; c < nch && ok; ++c) {
-                    if (c + 2 < nch) ok = issue_s(g + c + 2, c + 2, it);
-                    if (ok) ok = issue_pv(g + c, c, it);
+                MaskRow mr;
+                const int64_t nch = (item_keys<FUSED, MQ>(p, item, false, mr, lane) + 127) / 128;
+                if (lane == 0) {
+                    // S of chunks 0 and 1, then for every chunk c the S of chunk c+2 (its slot
+                    // frees as soon as the softmax has read chunk c) before the P.V of chunk c
+                    for (int64_t c = 0; c < nch && c < 2 && ok; ++c) ok = issue_s(g + c, c, it);
+                    for (int64_t c = 0; c < nch && ok; ++c) {
+                        if (c + 2 < nch) ok = issue_s(g + c + 2, c + 2, it);
+                        if (ok) ok = issue_pv(g + c, c, it);
+                    }
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
                 g += nch;
             }
             // drain: every MMA issued has completed before TMEM is freed
-            ptx::mma_commit(BAR(C::B_DRAIN));
-            bounded_wait(BAR(C::B_DRAIN), 0u, abort_flag, /*honour_abort=*/false);
+            if (lane == 0) {
+                ptx::mma_commit(BAR(C::B_DRAIN));
+                bounded_wait(BAR(C::B_DRAIN), 0u, abort_flag, /*honour_abort=*/false);
+            }
         }
         __syncwarp();
     } else {
@@ -439,7 +460,11 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
         for (int64_t item = blockIdx.x; item < p.items; item += gridDim.x) {
             const int64_t bh = item / p.QB;
             const int64_t qb = item - bh * p.QB;
-            const int64_t cnt = item_count(p, item, false);
+            int64_t cnt;
+            {
+                MaskRow mr;
+                cnt = item_keys<FUSED, MQ>(p, item, false, mr, lane);
+            }
             const int64_t nch = (cnt + 127) / 128;
             float mref = -INFINITY;  // reference of this row (log2 units of the scaled scores)
             float lsum = 0.f;        // this half's partial row sum

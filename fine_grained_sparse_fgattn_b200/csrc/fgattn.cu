@@ -177,13 +177,13 @@ bool encode_maps_uncached(fgattn::FwdParams& prm, const void* q, const Strides& 
     return true;
 }
 
-template <int D, int MQ, bool GATHER, bool STRIDED>
+template <int D, int MQ, bool GATHER, bool STRIDED, bool FUSED>
 fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
                          const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows,
                          cudaStream_t stream) {
     using C = fgattn::FwdCfg<D, MQ, GATHER>;
     if (!encode_maps<STRIDED>(prm, q, qs, k, ks, v, vs, B, H, D, k_rows, MQ)) return FGATTN_ERR_CUDA;
-    auto kernel = fgattn::fgattn_fwd_kernel<D, MQ, GATHER, STRIDED>;
+    auto kernel = fgattn::fgattn_fwd_kernel<D, MQ, GATHER, STRIDED, FUSED>;
     // Request enough shared memory that exactly one block is resident per SM:
     // the grid is persistent (one block per SM, static round-robin over work).
     const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;
@@ -211,12 +211,12 @@ fgattn_status launch_fwd(fgattn::FwdParams& prm, const void* q, const Strides& q
 }
 
 // Query-major kernel (128-row query blocks): M = 128 lists and dense runs.
-template <int D, bool GATHER, bool STRIDED>
+template <int D, bool GATHER, bool STRIDED, bool FUSED>
 fgattn_status launch_qm(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
                         const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows, cudaStream_t stream) {
     using C = fgattn::QmCfg<D, GATHER>;
     if (!encode_maps<STRIDED>(prm, q, qs, k, ks, v, vs, B, H, D, k_rows, C::MQ)) return FGATTN_ERR_CUDA;
-    auto kernel = fgattn::fgattn_fwd_qm_kernel<D, GATHER, STRIDED>;
+    auto kernel = fgattn::fgattn_fwd_qm_kernel<D, GATHER, STRIDED, FUSED>;
     const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;  // one block per SM
     // the attribute is per function and device: set and checked once per device
     static bool configured[kMaxConfigDevices] = {};
@@ -238,47 +238,46 @@ fgattn_status launch_qm(fgattn::FwdParams& prm, const void* q, const Strides& qs
     return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
 }
 
-template <int D, bool GATHER, bool STRIDED>
+template <int D, bool GATHER, bool STRIDED, bool FUSED>
 fgattn_status dispatch_m(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
                          const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows, int64_t M,
                          cudaStream_t s) {
-    // 128-row query blocks (M = 128 lists, or a dense run of any M: every key is kept,
-    // so the result does not depend on M) go to the query-major kernel.
-    if (M == 128 || prm.kept_idx == nullptr) {
+    // 128-row query blocks (M = 128 lists or masks, or a dense run of any M: every key
+    // is kept, so the result does not depend on M) go to the query-major kernel.
+    if (M == 128 || (prm.kept_idx == nullptr && prm.mask == nullptr)) {
         prm.QB = (prm.L + 127) / 128;
         prm.items = B * H * prm.QB;
         // the query-major softmax needs a non-zero scale: a scale of magnitude below
         // 1e-30 (log2 units) gives the same probabilities (every score maps to 2^0)
         if (std::fabs(prm.scale_log2) < 1e-30f) prm.scale_log2 = prm.scale_log2 < 0.f ? -1e-30f : 1e-30f;
-        return launch_qm<D, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
+        return launch_qm<D, GATHER, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
     }
     switch (M) {
-        case 16: return launch_fwd<D, 16, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
-        case 32: return launch_fwd<D, 32, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
-        case 64: return launch_fwd<D, 64, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
-        default: return launch_fwd<D, 128, GATHER, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
+        case 16: return launch_fwd<D, 16, GATHER, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
+        case 32: return launch_fwd<D, 32, GATHER, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
+        default: return launch_fwd<D, 64, GATHER, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, s);
     }
 }
 
-template <bool STRIDED>
+template <bool STRIDED, bool FUSED = false>
 fgattn_status dispatch(fgattn::FwdParams& prm, const void* q, const Strides& qs, const void* k, const Strides& ks,
                        const void* v, const Strides& vs, int64_t B, int64_t H, int64_t k_rows, int64_t d, int64_t M,
                        bool gather, cudaStream_t s) {
     if (d == 128)
-        return gather ? dispatch_m<128, true, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
-                      : dispatch_m<128, false, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
+        return gather ? dispatch_m<128, true, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
+                      : dispatch_m<128, false, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
     if (d == 96)
-        return gather ? dispatch_m<96, true, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
-                      : dispatch_m<96, false, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
-    return gather ? dispatch_m<64, true, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
-                  : dispatch_m<64, false, STRIDED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
+        return gather ? dispatch_m<96, true, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
+                      : dispatch_m<96, false, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
+    return gather ? dispatch_m<64, true, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s)
+                  : dispatch_m<64, false, STRIDED, FUSED>(prm, q, qs, k, ks, v, vs, B, H, k_rows, M, s);
 }
 
 // Shared by fgattn_forward (contiguous [B][H][L][d]) and fgattn_forward_strided.
 fgattn_status forward_impl(const void* q, const Strides& qs, const void* k, const Strides& ks, const void* v,
                            const Strides& vs, const int32_t* kept_idx, const int32_t* kept_cnt, int64_t cap, int64_t B,
                            int64_t H, int64_t L, int64_t d, int64_t M, int64_t N, float scale, void* out,
-                           const Strides& os, float* lse, fgattn_stream_t stream) {
+                           const Strides& os, float* lse, fgattn_stream_t stream, const uint32_t* mask = nullptr) {
     if (!q || !k || !v || !out) return FGATTN_ERR_INVALID_ARG;
     if (kept_idx && !kept_cnt) return FGATTN_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || L < 1 || M < 1 || N < 1 || d < 1) return FGATTN_ERR_INVALID_ARG;
@@ -307,6 +306,15 @@ fgattn_status forward_impl(const void* q, const Strides& qs, const void* k, cons
     fgattn::FwdParams prm;
     prm.kept_idx = kept_idx;
     prm.kept_cnt = kept_cnt;
+    prm.mask = nullptr;
+    prm.mask_w = prm.mask_g = prm.mask_n = 0;
+    if (mask) {  // fused kernels: the mask is read in place of kept lists
+        const int64_t Ng = N > L ? L : N;  // one key group either way when N > L
+        prm.mask = mask;
+        prm.mask_n = Ng;
+        prm.mask_g = (L + Ng - 1) / Ng;
+        prm.mask_w = (prm.mask_g + 31) / 32;
+    }
     prm.out = static_cast<__nv_bfloat16*>(out);
     prm.lse = lse;
     prm.cap = kept_idx ? cap : L;
@@ -321,7 +329,7 @@ fgattn_status forward_impl(const void* q, const Strides& qs, const void* k, cons
     prm.o_sb = os.s[0], prm.o_sh = os.s[1], prm.o_sl = os.s[2];
     // Lists of whole 16-key runs (N a multiple of 16) load as TMA tiles: tile layout.
     // Anything else is gathered row by row: gather layout (more K producer warps).
-    const bool gather = kept_idx != nullptr && N % 16 != 0;
+    const bool gather = mask ? prm.mask_n % 16 != 0 : (kept_idx != nullptr && N % 16 != 0);
     // Contiguous [B][H][L][d] everywhere (strides of extent-1 dimensions aside): the
     // contiguous kernel.
     const Strides c = {{H * L * d, L * d, d}};
@@ -330,6 +338,10 @@ fgattn_status forward_impl(const void* q, const Strides& qs, const void* k, cons
     for (const Strides* t : {&qs, &ks, &vs, &os})
         for (int i = 0; i < 3; ++i) contiguous = contiguous && (extent[i] == 1 || t->s[i] == c.s[i]);
     cudaStream_t s = (cudaStream_t)stream;
+    if (mask) {
+        if (!contiguous) return FGATTN_ERR_UNSUPPORTED;
+        return dispatch<false, true>(prm, q, qs, k, ks, v, vs, B, H, k_rows, d, M, gather, s);
+    }
     if (contiguous) return dispatch<false>(prm, q, qs, k, ks, v, vs, B, H, k_rows, d, M, gather, s);
     return dispatch<true>(prm, q, qs, k, ks, v, vs, B, H, k_rows, d, M, gather, s);
 }
@@ -386,6 +398,19 @@ fgattn_status fgattn_forward_strided(const void* q, const int64_t* q_strides, co
     };
     const Strides qs = norm(q_strides), ks = norm(k_strides), vs = norm(v_strides), os = norm(out_strides);
     return forward_impl(q, qs, k, ks, v, vs, kept_idx, kept_cnt, cap, B, H, L, d, M, N, scale, out, os, lse, stream);
+}
+
+fgattn_status fgattn_masked_forward(const void* q, const void* k, const void* v, const uint32_t* mask, int64_t B,
+                                    int64_t H, int64_t L, int64_t d, int64_t M, int64_t N, float scale, void* out,
+                                    float* lse, fgattn_stream_t stream) {
+    if (!mask) return FGATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(mask) & 3u) return FGATTN_ERR_INVALID_ARG;
+    if (d < 1 || L < 1 || H < 1 || N < 1) return FGATTN_ERR_INVALID_ARG;
+    const int64_t Ng = N > L ? L : N;
+    const int64_t W = ((L + Ng - 1) / Ng + 31) / 32;
+    if (W > fgattn::kFusedMaxWords) return FGATTN_ERR_UNSUPPORTED;
+    const Strides c = {{H * L * d, L * d, d}};  // contiguous [B][H][L][d]
+    return forward_impl(q, c, k, c, v, c, nullptr, nullptr, L, B, H, L, d, M, N, scale, out, c, lse, stream, mask);
 }
 
 fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* bits) {

@@ -1,0 +1,112 @@
+// Fused mask expansion: the kept keys of one query block read straight from the
+// packed tile mask, by the warp that needs them, with no kept list in memory.
+//
+// The method skips M x N tiles ("FG-Attn: Leveraging Fine-Grained Sparse
+// Attention in Video Diffusion Models", Abstract); the mask holds one bit per
+// tile (row (b, h, qb) of W uint32 words, group g = bit g % 32 of word g / 32).
+// A block's key list is its kept groups in ascending order, each expanded to
+// its keys; the position of key j of the list is therefore fixed by the
+// number of kept groups before it.  A warp loads the row once per work item
+// (W <= 256 words: eight per lane), forces the block's diagonal groups and
+// drops bits past the last group (the same rules as the compaction kernel),
+// takes a prefix sum of the lanes' set-bit counts, and then finds the key at
+// any list position by itself: a five-step search over the lanes' prefix
+// counts, the lane's words by shuffle, and the n-th set bit of one word.  Every
+// role of the forward kernel that reads list entries does this for its own
+// entries, so the roles need no shared index structure.
+#pragma once
+
+#include <cstdint>
+
+namespace fgattn {
+
+constexpr int kFusedMaxWords = 256;  // mask words per row the fused expansion handles (G <= 8192)
+
+struct MaskRow {
+    static constexpr int WPL = kFusedMaxWords / 32;  // words per lane: lane l holds [8 l, 8 l + 8)
+    uint32_t w[WPL];
+    int32_t incl;  // kept groups in lanes 0 .. lane (inclusive prefix over the warp)
+    int32_t mine;  // kept groups in this lane's words
+    int64_t keys;  // kept keys of the row = the list length
+};
+
+// Warp-collective: row `item` (= (b * H + h) * QB + qb) of the mask.  mq = query
+// rows per block, n = keys per group, g = groups per row, wds = words per row.
+__device__ __forceinline__ void mask_row_load(MaskRow& r, const uint32_t* mask, int64_t item, int64_t qb_count,
+                                              int64_t mq, int64_t n, int64_t g, int64_t wds, int64_t L, int lane) {
+    const int64_t qb = item % qb_count;
+    const uint32_t* row = mask + item * wds;
+    const int64_t glo = (qb * mq) / n;                               // diagonal groups [glo, ghi]
+    const int64_t ghi = ((qb * mq + mq < L ? qb * mq + mq : L) - 1) / n;
+    int mine = 0;
+#pragma unroll
+    for (int i = 0; i < MaskRow::WPL; ++i) {
+        const int64_t wi = (int64_t)lane * MaskRow::WPL + i;
+        uint32_t x = wi < wds ? __ldg(row + wi) : 0u;
+        const int64_t g0 = wi * 32;
+        const int64_t lo = glo - g0 > 0 ? glo - g0 : 0;
+        const int64_t hi = ghi - g0 < 31 ? ghi - g0 : 31;
+        if (lo <= hi) {
+            const int nb = (int)(hi - lo + 1);
+            x |= (nb == 32 ? 0xffffffffu : ((1u << nb) - 1u)) << lo;
+        }
+        const int64_t valid = g - g0;  // groups of this word that exist
+        if (valid <= 0)
+            x = 0u;
+        else if (valid < 32)
+            x &= (1u << valid) - 1u;
+        r.w[i] = x;
+        mine += __popc(x);
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    r.incl = incl;
+    r.mine = mine;
+    const int64_t total = __shfl_sync(0xffffffffu, incl, 31);
+    // is the last group (which may hold fewer than n keys) kept?
+    const int64_t wl = (g - 1) / 32;
+    const int owner = (int)(wl / MaskRow::WPL), idx = (int)(wl % MaskRow::WPL);
+    uint32_t mine_w = 0u;
+#pragma unroll
+    for (int i = 0; i < MaskRow::WPL; ++i)
+        if (i == idx) mine_w = r.w[i];
+    const uint32_t lw = __shfl_sync(0xffffffffu, mine_w, owner);
+    const bool last_kept = (lw >> ((g - 1) % 32)) & 1u;
+    const int64_t lastlen = L - (g - 1) * n;
+    r.keys = total * n - (last_kept ? n - lastlen : 0);
+}
+
+// Warp-collective: the key at list position pos (each lane its own pos); 0 for
+// positions past the list (their scores are masked by the softmax).
+__device__ __forceinline__ int32_t mask_row_key(const MaskRow& r, int64_t pos, int64_t n, int lane) {
+    const bool inside = pos >= 0 && pos < r.keys;
+    const int32_t rank = inside ? (int32_t)(pos / n) : 0;  // which kept group
+    const int64_t off = inside ? pos - (int64_t)rank * n : 0;
+    // first lane whose inclusive count exceeds rank
+    int j = 0;
+#pragma unroll
+    for (int step = 16; step > 0; step >>= 1) {
+        const int cand = __shfl_sync(0xffffffffu, r.incl, j + step - 1);
+        if (cand <= rank) j += step;
+    }
+    int rr = rank - (__shfl_sync(0xffffffffu, r.incl, j) - __shfl_sync(0xffffffffu, r.mine, j));
+    int32_t grp = 0;
+    bool found = false;
+#pragma unroll
+    for (int i = 0; i < MaskRow::WPL; ++i) {
+        const uint32_t wv = __shfl_sync(0xffffffffu, r.w[i], j);
+        const int c = __popc(wv);
+        if (!found && rr < c) {
+            grp = (j * MaskRow::WPL + i) * 32 + (int)__fns(wv, 0u, rr + 1);
+            found = true;
+        }
+        if (!found) rr -= c;
+    }
+    return inside ? (int32_t)((int64_t)grp * n + off) : 0;
+}
+
+}  // namespace fgattn

@@ -135,6 +135,29 @@ fgattn_status fgattn_forward_strided(const void* q, const int64_t* q_strides, co
                                      float* lse, fgattn_stream_t stream);
 
 /*
+ * Tile-sparse attention forward straight from the mask, in one kernel: the
+ * mask compaction fused into the forward ("FG-Attn ...", Abstract: the M x N
+ * tiles are skipped at that granularity; the mask is the tile list).  Every
+ * warp of the kernel that needs kept keys reads its query block's mask row and
+ * expands it itself (diagonal rule and ragged ends as fgattn_compact_mask), so
+ * no kept list is written to or read from memory and nothing is allocated.
+ *   q, k, v   in   device bf16 [B][H][L][d], contiguous
+ *   mask      in   device uint32 [B][H][QB][W] (layout as above)
+ *   out       out  device bf16 [B][H][L][d]
+ *   lse       out  device fp32 [B][H][L], may be NULL
+ * Results equal fgattn_compact_mask followed by fgattn_forward, bit for bit
+ * (same kernels, same key order).  Supported: as fgattn_forward, and
+ * W = ceil(ceil(L / N) / 32) <= 256 mask words per query block (for example
+ * N = 16 up to L = 131072, N = 1 up to L = 8192); larger rows return
+ * UNSUPPORTED (use fgattn_compact_mask + fgattn_forward).
+ * Errors: INVALID_ARG (also a NULL or misaligned mask), UNSUPPORTED, CUDA;
+ * device-side problems as for fgattn_forward.
+ */
+fgattn_status fgattn_masked_forward(const void* q, const void* k, const void* v, const uint32_t* mask, int64_t B,
+                                    int64_t H, int64_t L, int64_t d, int64_t M, int64_t N, float scale, void* out,
+                                    float* lse, fgattn_stream_t stream);
+
+/*
  * Synchronise `stream`, then report (and, if clear != 0, reset) the device
  * error bits (FGATTN_DEVERR_*) recorded on the current device since the last
  * clear.  *bits may be NULL.  Returns DEVICE if any bit is set, CUDA if the

@@ -110,6 +110,31 @@ def test_compact_rejects(kw, status):
     assert _cmp(**kw) == status
 
 
+def _mfwd(**kw):
+    a = dict(q=P, k=P, v=P, mask=P, B=1, H=1, L=64, d=128, M=64, N=16, scale=0.1, out=P, lse=P)
+    a.update(kw)
+    return F._lib.fgattn_masked_forward(a["q"], a["k"], a["v"], a["mask"], a["B"], a["H"], a["L"], a["d"], a["M"],
+                                        a["N"], a["scale"], a["out"], a["lse"], None)
+
+
+@no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(mask=None), F.ERR_INVALID_ARG),
+    (dict(mask=P + 2), F.ERR_INVALID_ARG),
+    (dict(q=None), F.ERR_INVALID_ARG),
+    (dict(L=0), F.ERR_INVALID_ARG),
+    (dict(N=0), F.ERR_INVALID_ARG),
+    (dict(q=P + 8), F.ERR_INVALID_ARG),
+    (dict(d=80), F.ERR_UNSUPPORTED),
+    (dict(M=48), F.ERR_UNSUPPORTED),
+    # rows of more than 256 mask words (here 32760 groups of one key: 1024 words)
+    (dict(L=32760, N=1), F.ERR_UNSUPPORTED),
+    (dict(L=8192 * 16 + 16, N=16), F.ERR_UNSUPPORTED),
+])
+def test_masked_forward_rejects(kw, status):
+    assert _mfwd(**kw) == status
+
+
 @no_gpu
 def test_valid_call_without_gpu_reports_cuda_error():
     # All arguments valid, so the launch is attempted; with no device it fails cleanly.
