@@ -272,15 +272,24 @@ __device__ __forceinline__ int4 fetch_idx(const int32_t* lst, int64_t cnt, int64
 
 // Fused kernels: list entries 4*lane .. 4*lane+3 of chunk c from the mask row
 // (warp-collective; every lane of the warp calls it).
-__device__ __forceinline__ int4 fused_idx4(const MaskRow& mr, int64_t n, int64_t c, int lane4, int lane) {
+__device__ __forceinline__ int4 fused_idx4(const MaskRow& mr, int64_t c, int lane4, int lane) {
     const int64_t j0 = c * 128 + 4 * lane4;
-    if (n % 4 == 0) {  // four consecutive keys of one group
-        const int32_t k = mask_row_key(mr, j0, n, lane);
+    if ((mr.n & 3) == 0) {  // four consecutive keys of one group
+        const int32_t k = mask_row_key(mr, j0, lane);
         return make_int4(j0 < mr.keys ? k : 0, j0 + 1 < mr.keys ? k + 1 : 0, j0 + 2 < mr.keys ? k + 2 : 0,
                          j0 + 3 < mr.keys ? k + 3 : 0);
     }
-    return make_int4(mask_row_key(mr, j0, n, lane), mask_row_key(mr, j0 + 1, n, lane),
-                     mask_row_key(mr, j0 + 2, n, lane), mask_row_key(mr, j0 + 3, n, lane));
+    // four separate searches, one copy of the search code (kept small for the instruction cache)
+    int4 e = make_int4(0, 0, 0, 0);
+#pragma unroll 1
+    for (int x = 0; x < 4; ++x) {
+        const int32_t k = mask_row_key(mr, j0 + x, lane);
+        e.x = x == 0 ? k : e.x;
+        e.y = x == 1 ? k : e.y;
+        e.z = x == 2 ? k : e.z;
+        e.w = x == 3 ? k : e.w;
+    }
+    return e;
 }
 
 // Kept keys of work item `item`: from kept_cnt, L for a dense run, or the mask
@@ -407,7 +416,7 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
             const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
             auto fetch4 = [&](int64_t c) -> int4 {  // this lane's four entries of chunk c (-1: none)
                 if constexpr (FUSED) {
-                    const int4 e = fused_idx4(mr, p.mask_n, c, g4, lane);  // every lane takes part
+                    const int4 e = fused_idx4(mr, c, g4, lane);  // every lane takes part
                     return issuer ? e : make_int4(-1, -1, -1, -1);
                 } else {
                     return issuer ? fetch_idx(lst, cnt, c, g4) : make_int4(-1, -1, -1, -1);
@@ -437,15 +446,28 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
             }
             constexpr int PF = 4;  // index prefetch distance in chunks (the lists live in HBM)
             int4 ring[PF];
+            // fused kernels: no ring, the next chunk's entries are computed one chunk ahead (one
+            // copy of the expansion code per producer keeps the instruction cache warm)
+            int4 nxt = make_int4(-1, -1, -1, -1);
+            if constexpr (FUSED) {
+                if (nch > 0) nxt = fetch4(0);
+            } else {
 #pragma unroll
-            for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch4(i) : make_int4(-1, -1, -1, -1);
+                for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch4(i) : make_int4(-1, -1, -1, -1);
+            }
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
                 const int st = (int)(gc % NK);
-                const int4 cur = ring[0];
+                int4 cur;
+                if constexpr (FUSED) {
+                    cur = nxt;
+                    if (c + 1 < nch) nxt = fetch4(c + 1);
+                } else {
+                    cur = ring[0];
 #pragma unroll
-                for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
-                ring[PF - 1] = c + PF < nch ? fetch4(c + PF) : make_int4(-1, -1, -1, -1);
+                    for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
+                    ring[PF - 1] = c + PF < nch ? fetch4(c + PF) : make_int4(-1, -1, -1, -1);
+                }
                 const bool okw =
                     gc < NK || bounded_wait(BAR(C::B_KEMPTY + st), (uint32_t)((gc / NK - 1) & 1), abort_flag);
                 if (!__all_sync(0xffffffffu, okw)) {
@@ -522,7 +544,7 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
             auto fetch1 = [&](int64_t c) -> int32_t {
                 const int64_t j = c * 128 + vw * 32 + lane;
                 if constexpr (FUSED) {
-                    const int32_t k = mask_row_key(mr, j, p.mask_n, lane);  // every lane takes part
+                    const int32_t k = mask_row_key(mr, j, lane);  // every lane takes part
                     return j >= cnt ? -1 : k;
                 } else {
                     if (j >= cnt) return -1;  // past the list
@@ -531,15 +553,26 @@ __global__ void __launch_bounds__(FwdCfg<D, MQ, GATHER>::THREADS, 1)
             };
             constexpr int PF = 4;
             int32_t ring[PF];
+            int32_t nxt = -1;  // fused kernels: one chunk ahead, no ring
+            if constexpr (FUSED) {
+                if (nch > 0) nxt = fetch1(0);
+            } else {
 #pragma unroll
-            for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch1(i) : -1;
+                for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch1(i) : -1;
+            }
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
                 const int st = (int)(gc % NV);
-                int32_t idx = ring[0];
+                int32_t idx;
+                if constexpr (FUSED) {
+                    idx = nxt;
+                    if (c + 1 < nch) nxt = fetch1(c + 1);
+                } else {
+                    idx = ring[0];
 #pragma unroll
-                for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
-                ring[PF - 1] = c + PF < nch ? fetch1(c + PF) : -1;
+                    for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
+                    ring[PF - 1] = c + PF < nch ? fetch1(c + PF) : -1;
+                }
                 // slot (gc % 2) is free once MMA2 of chunk gc-2 has completed
                 const bool okw =
                     gc < 2 || bounded_wait(BAR(C::B_ODONE + (int)(gc & 1)), (uint32_t)(((gc - 2) >> 1) & 1), abort_flag);

@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                 const int32_t* lst = p.kept_idx ? p.kept_idx + item * p.cap : nullptr;
                 auto fetch4 = [&](int64_t c) -> int4 {  // this lane's four entries of chunk c (-1: none)
                     if constexpr (FUSED) {
-                        const int4 e = fused_idx4(mr, p.mask_n, c, g4, lane);  // every lane takes part
+                        const int4 e = fused_idx4(mr, c, g4, lane);  // every lane takes part
                         return issuer ? e : make_int4(-1, -1, -1, -1);
                     } else {
                         return issuer ? fetch_idx(lst, cnt, c, g4) : make_int4(-1, -1, -1, -1);
@@ -198,15 +198,28 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
                 }
                 constexpr int PF = 4;  // index prefetch distance in chunks (the lists live in HBM)
                 int4 ring[PF];
+                // fused kernels: no ring, the next chunk's entries are computed one chunk ahead (one
+                // copy of the expansion code per producer keeps the instruction cache warm)
+                int4 nxt = make_int4(-1, -1, -1, -1);
+                if constexpr (FUSED) {
+                    if (nch > 0) nxt = fetch4(0);
+                } else {
 #pragma unroll
-                for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch4(i) : make_int4(-1, -1, -1, -1);
+                    for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch4(i) : make_int4(-1, -1, -1, -1);
+                }
                 for (int64_t c = 0; c < nch; ++c) {
                     const int64_t gc = g + c;
                     const int st = (int)(gc % NK);
-                    const int4 cur = ring[0];
+                    int4 cur;
+                    if constexpr (FUSED) {
+                        cur = nxt;
+                        if (c + 1 < nch) nxt = fetch4(c + 1);
+                    } else {
+                        cur = ring[0];
 #pragma unroll
-                    for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
-                    ring[PF - 1] = c + PF < nch ? fetch4(c + PF) : make_int4(-1, -1, -1, -1);
+                        for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
+                        ring[PF - 1] = c + PF < nch ? fetch4(c + PF) : make_int4(-1, -1, -1, -1);
+                    }
                     const bool okw =
                         gc < NK || bounded_wait(BAR(C::B_KEMPTY + st), (uint32_t)((gc / NK - 1) & 1), abort_flag);
                     if (!__all_sync(0xffffffffu, okw)) {
@@ -284,7 +297,7 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
             auto fetch1 = [&](int64_t c) -> int32_t {
                 const int64_t j = c * 128 + vw * 32 + lane;
                 if constexpr (FUSED) {
-                    const int32_t k = mask_row_key(mr, j, p.mask_n, lane);  // every lane takes part
+                    const int32_t k = mask_row_key(mr, j, lane);  // every lane takes part
                     return j >= cnt ? -1 : k;
                 } else {
                     if (j >= cnt) return -1;  // past the list
@@ -293,15 +306,26 @@ __global__ void __launch_bounds__(512, 1) fgattn_fwd_qm_kernel(const __grid_cons
             };
             constexpr int PF = 4;
             int32_t ring[PF];
+            int32_t nxt = -1;  // fused kernels: one chunk ahead, no ring
+            if constexpr (FUSED) {
+                if (nch > 0) nxt = fetch1(0);
+            } else {
 #pragma unroll
-            for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch1(i) : -1;
+                for (int i = 0; i < PF; ++i) ring[i] = i < nch ? fetch1(i) : -1;
+            }
             for (int64_t c = 0; c < nch; ++c) {
                 const int64_t gc = g + c;
                 const int st = (int)(gc % NV);
-                int32_t idx = ring[0];
+                int32_t idx;
+                if constexpr (FUSED) {
+                    idx = nxt;
+                    if (c + 1 < nch) nxt = fetch1(c + 1);
+                } else {
+                    idx = ring[0];
 #pragma unroll
-                for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
-                ring[PF - 1] = c + PF < nch ? fetch1(c + PF) : -1;
+                    for (int i = 0; i < PF - 1; ++i) ring[i] = ring[i + 1];
+                    ring[PF - 1] = c + PF < nch ? fetch1(c + PF) : -1;
+                }
                 const bool okw = gc < 2 || bounded_wait(BAR(C::B_ODONE + (int)(gc & 1)),
                                                         (uint32_t)(((gc - 2) >> 1) & 1), abort_flag);
                 if (!__all_sync(0xffffffffu, okw)) {
