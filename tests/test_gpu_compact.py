@@ -68,6 +68,10 @@ def test_workload_masks_full_arrays(oracle, name, N, sp):
     (1, 16, 1, 0.0), (1, 16, 8, 1.0), (17, 16, 1, 0.5), (100, 16, 3, 0.0), (100, 16, 3, 1.0),
     (257, 64, 7, 0.3), (1000, 128, 1, 0.2), (4097, 64, 33, 0.5), (64, 64, 100, 0.5), (33, 1, 1, 0.5),
     (2048, 32, 2, 0.05), (5000, 16, 1, 0.9),
+    # rows of more than 64 words (eight warps per row): three batches over eight warps,
+    # a ragged last group with int4 stores, all ones / all zeros, many batches per warp
+    (2080, 64, 1, 0.3), (9002, 64, 4, 0.4), (5000, 16, 1, 1.0), (4200, 64, 2, 0.0), (40000, 128, 1, 0.3),
+    (65 * 32 * 3 + 5, 16, 3, 0.5),
 ])
 def test_edge_masks(oracle, L, M, N, density):
     QB, G = -(-L // M), -(-L // N)
