@@ -5,7 +5,8 @@ and by the benchmark's CPU-baseline leg, never by the product path.
 
 The oracle evaluates tile-sparse softmax attention by its definition in double
 precision ("FG-Attn: Leveraging Fine-Grained Sparse Attention in Video
-Diffusion Models", Abstract: skipped M x N score tiles count as -inf).
+Diffusion Models", Abstract: skipped M x N score tiles count as -inf), and the
+gradients of that definition with respect to q, k and v (backward).
 Parity of every function here is pinned by tests/test_oracle.py against
 library routines (torch float64 softmax), brute force and closed forms.
 """
@@ -52,6 +53,9 @@ class Oracle:
         self._lib.oracle_attention.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64,
                                                ctypes.c_double, p, i64, p, p, ctypes.c_int]
         self._lib.oracle_attention.restype = ctypes.c_int
+        self._lib.oracle_attention_backward.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, i64,
+                                                        ctypes.c_double, p, p, p, ctypes.c_int]
+        self._lib.oracle_attention_backward.restype = ctypes.c_int
 
     # ------------------------------------------------------------------
     def compact(self, mask: np.ndarray, B: int, H: int, L: int, M: int, N: int, cap: Optional[int] = None):
@@ -94,6 +98,29 @@ class Oracle:
         if st != 0:
             raise RuntimeError(f"oracle_attention failed ({st})")
         return out, lse
+
+
+    def backward(self, q, k, v, dout, mask: np.ndarray, M: int, N: int, scale: float, nthreads: int = 0):
+        """Gradients of the forward with respect to q, k and v for the upstream gradient
+        dout (bf16 like q, k, v) of out, every head.  Returns float64 arrays
+        (dq, dk, dv), each [B, H, L, d]."""
+        qb16, kb16, vb16, db16 = (_bits(x) for x in (q, k, v, dout))
+        B, H, L, d = qb16.shape
+        mask = np.ascontiguousarray(mask, dtype=np.uint32)
+        QB, G = -(-L // M), -(-L // N)
+        assert mask.size == B * H * QB * (-(-G // 32)), "mask has the wrong size"
+        dq = np.empty((B, H, L, d), dtype=np.float64)
+        dk = np.empty_like(dq)
+        dv = np.empty_like(dq)
+        if nthreads <= 0:
+            nthreads = os.cpu_count() or 1
+        st = self._lib.oracle_attention_backward(qb16.ctypes.data, kb16.ctypes.data, vb16.ctypes.data,
+                                                 db16.ctypes.data, mask.ctypes.data, B, H, L, d, M, N,
+                                                 float(scale), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data,
+                                                 int(nthreads))
+        if st != 0:
+            raise RuntimeError(f"oracle_attention_backward failed ({st})")
+        return dq, dk, dv
 
 
 def _bits(x) -> np.ndarray:

@@ -29,6 +29,9 @@
  *   - keys >= L do not exist; the last group holds L - (G-1)*N keys;
  *     query rows >= L are neither computed nor written.
  *
+ * The backward pass (oracle_attention_backward, at the end of this file) is the
+ * plain gradient of the same definition, also in double precision.
+ *
  * Build with any C99 compiler:  cc -O2 -shared -fPIC -pthread fgattn_oracle.c
  * (no -ffast-math: the sums must be evaluated in program order).
  *
@@ -234,6 +237,156 @@ int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, co
         int started = 0;
         for (int w = 0; w < nthreads; ++w) {
             if (pthread_create(&tid[w], NULL, worker, &jobs[w]) != 0) { status = -3; break; }
+            ++started;
+        }
+        for (int w = 0; w < started; ++w) pthread_join(tid[w], NULL);
+        for (int w = 0; w < nthreads && !status; ++w) status = jobs[w].status;
+    }
+    free(jobs);
+    free(tid);
+    return status;
+}
+
+/*
+ * Backward pass (gradients of the forward above), evaluated in double precision
+ * by the definition, per (b, h) head: with p_ij = exp(s_ij - m_i) / l_i for the
+ * kept scores (0 for skipped ones) and the upstream gradient dO of out,
+ *
+ *   dP_ij = dO_i . v_j                 D_i   = sum_j p_ij dP_ij  (= dO_i . out_i)
+ *   dS_ij = p_ij (dP_ij - D_i)
+ *   dq_i  = scale * sum_j dS_ij k_j    dk_j  = scale * sum_i dS_ij q_i
+ *   dv_j  = sum_i p_ij dO_i
+ *
+ * (the chain rule through s = scale * q . k, the softmax and out = P v; a
+ * skipped score has p = 0 and contributes to no gradient).  q, k, v, dout:
+ * bf16 bit patterns [B][H][L][d]; dq, dk, dv: double [B][H][L][d].
+ */
+typedef struct {
+    const uint16_t *q, *k, *v, *dout;
+    const uint32_t* mask;
+    int64_t B, H, L, d, M, N;
+    double scale;
+    double *dq, *dk, *dv;
+    int64_t first, last; /* this worker's share of heads */
+    int status;
+} bjob_t;
+
+static int backward_head(const bjob_t* J, int64_t bh) {
+    const int64_t L = J->L, d = J->d, M = J->M, N = J->N;
+    const int64_t QB = (L + M - 1) / M;
+    const int64_t G = (L + N - 1) / N;
+    const int64_t W = (G + 31) / 32;
+    const uint16_t* Q = J->q + bh * L * d;
+    const uint16_t* K = J->k + bh * L * d;
+    const uint16_t* V = J->v + bh * L * d;
+    const uint16_t* DO = J->dout + bh * L * d;
+    double* dq = J->dq + bh * L * d;
+    double* dk = J->dk + bh * L * d;
+    double* dv = J->dv + bh * L * d;
+    double* s = (double*)malloc((size_t)L * sizeof(double));
+    double* dp = (double*)malloc((size_t)L * sizeof(double));
+    char* kept = (char*)malloc((size_t)G);
+    if (!s || !dp || !kept) { free(s); free(dp); free(kept); return -2; }
+    for (int64_t x = 0; x < L * d; ++x) { dk[x] = 0.0; dv[x] = 0.0; }
+    for (int64_t i = 0; i < L; ++i) {
+        const int64_t qb = i / M;
+        const uint32_t* mrow = J->mask + (bh * QB + qb) * W;
+        for (int64_t g = 0; g < G; ++g) kept[g] = (char)tile_kept(mrow, qb, g, L, M, N);
+        /* probabilities of row i */
+        double m = -INFINITY;
+        for (int64_t j = 0; j < L; ++j) {
+            if (!kept[j / N]) { s[j] = -INFINITY; continue; }
+            double acc = 0.0;
+            for (int64_t t = 0; t < d; ++t) acc += bf16_to_double(Q[i * d + t]) * bf16_to_double(K[j * d + t]);
+            s[j] = J->scale * acc;
+            if (s[j] > m) m = s[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < L; ++j) l += exp(s[j] - m);
+        /* dP_ij and D_i */
+        double D = 0.0;
+        for (int64_t j = 0; j < L; ++j) {
+            if (s[j] == -INFINITY) { dp[j] = 0.0; continue; }
+            double acc = 0.0;
+            for (int64_t t = 0; t < d; ++t) acc += bf16_to_double(DO[i * d + t]) * bf16_to_double(V[j * d + t]);
+            dp[j] = acc;
+#if ORACLE_MUTANT == 11 /* planted: dv from unnormalised probabilities (no division by l) */
+            const double p = exp(s[j] - m);
+#else
+            const double p = exp(s[j] - m) / l;
+#endif
+            D += p * acc;
+        }
+        for (int64_t t = 0; t < d; ++t) dq[i * d + t] = 0.0;
+        for (int64_t j = 0; j < L; ++j) {
+            if (s[j] == -INFINITY) continue;
+#if ORACLE_MUTANT == 11
+            const double p = exp(s[j] - m);
+#else
+            const double p = exp(s[j] - m) / l;
+#endif
+#if ORACLE_MUTANT == 9 /* planted: the -D_i term dropped */
+            const double ds = p * dp[j];
+#else
+            const double ds = p * (dp[j] - D);
+#endif
+            for (int64_t t = 0; t < d; ++t) {
+#if ORACLE_MUTANT == 12 /* planted: dq accumulates the query instead of the key */
+                dq[i * d + t] += J->scale * ds * bf16_to_double(Q[i * d + t]);
+#else
+                dq[i * d + t] += J->scale * ds * bf16_to_double(K[j * d + t]);
+#endif
+#if ORACLE_MUTANT == 10 /* planted: dk without the scale */
+                dk[j * d + t] += ds * bf16_to_double(Q[i * d + t]);
+#else
+                dk[j * d + t] += J->scale * ds * bf16_to_double(Q[i * d + t]);
+#endif
+                dv[j * d + t] += p * bf16_to_double(DO[i * d + t]);
+            }
+        }
+    }
+    free(s);
+    free(dp);
+    free(kept);
+    return 0;
+}
+
+static void* bworker(void* arg) {
+    bjob_t* J = (bjob_t*)arg;
+    for (int64_t bh = J->first; bh < J->last; ++bh) {
+        int st = backward_head(J, bh);
+        if (st) { J->status = st; break; }
+    }
+    return NULL;
+}
+
+/* Gradients dq, dk, dv of every head (see above).  Returns 0 on success. */
+int oracle_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                              const uint32_t* mask, int64_t B, int64_t H, int64_t L, int64_t d, int64_t M,
+                              int64_t N, double scale, double* dq, double* dk, double* dv, int nthreads) {
+    const int64_t heads = B * H;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > heads) nthreads = (int)(heads > 0 ? heads : 1);
+    bjob_t* jobs = (bjob_t*)calloc((size_t)nthreads, sizeof(bjob_t));
+    pthread_t* tid = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return -2; }
+    for (int w = 0; w < nthreads; ++w) {
+        bjob_t* J = &jobs[w];
+        J->q = q; J->k = k; J->v = v; J->dout = dout; J->mask = mask;
+        J->B = B; J->H = H; J->L = L; J->d = d; J->M = M; J->N = N; J->scale = scale;
+        J->dq = dq; J->dk = dk; J->dv = dv;
+        J->first = heads * w / nthreads;
+        J->last = heads * (w + 1) / nthreads;
+        J->status = 0;
+    }
+    int status = 0;
+    if (nthreads == 1) {
+        bworker(&jobs[0]);
+        status = jobs[0].status;
+    } else {
+        int started = 0;
+        for (int w = 0; w < nthreads; ++w) {
+            if (pthread_create(&tid[w], NULL, bworker, &jobs[w]) != 0) { status = -3; break; }
             ++started;
         }
         for (int w = 0; w < started; ++w) pthread_join(tid[w], NULL);

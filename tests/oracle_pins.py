@@ -212,6 +212,62 @@ def check_compaction_invariants(oracle):
             assert (rep == forced).all()
 
 
+# ---------------------------------------------------------------------------
+# Backward pass: the gradients of the same definition with respect to q, k and v.
+def _autograd(q, k, v, dout, keep, scale):
+    """torch float64 autograd of masked softmax attention with loss = sum(out * dout)."""
+    qd, kd, vd = (torch.from_numpy(_f64(x)).requires_grad_(True) for x in (q, k, v))
+    s = scale * (qd @ kd.T)
+    s = s.masked_fill(~torch.from_numpy(keep), float("-inf"))
+    out = torch.softmax(s, dim=-1) @ vd
+    (out * torch.from_numpy(_f64(dout))).sum().backward()
+    return qd.grad.numpy(), kd.grad.numpy(), vd.grad.numpy()
+
+
+def check_backward_matches_torch_autograd(oracle):
+    """All tiles kept and random tiles (per-score -inf mask built with loops, plus the
+    diagonal rule): the oracle's gradients equal torch float64 autograd."""
+    cases = [(40, 8, 16, 40, 1.0), (37, 8, 16, 3, 0.3), (64, 16, 32, 8, 0.4), (50, 8, 16, 1, 0.2)]
+    for ci, (L, d, M, N, dens) in enumerate(cases):
+        q, k, v = W.random_qkv(1, 2, L, d, 50 + ci)
+        dout, _, _ = W.random_qkv(1, 2, L, d, 60 + ci)
+        QB, G = -(-L // M), -(-L // N)
+        tiles = np.ones((1, 2, QB, G), dtype=bool) if dens >= 1.0 else W.random_tiles(1, 2, QB, G, dens, 70 + ci)
+        scale = 0.31
+        dq, dk, dv = oracle.backward(q, k, v, dout, W.pack_tiles(tiles), M, N, scale, nthreads=2)
+        for h in range(2):
+            keep = _dense_kept(tiles[0, h], L, M, N)
+            rq, rk, rv = _autograd(q[0, h], k[0, h], v[0, h], dout[0, h], keep, scale)
+            for name, a, b in (("dq", dq[0, h], rq), ("dk", dk[0, h], rk), ("dv", dv[0, h], rv)):
+                assert np.abs(a - b).max() < TOL, f"{name} differs from autograd (case {ci})"
+
+
+def check_backward_invariants(oracle):
+    """sum_j dS_ij = 0 for every row, hence sum over keys of dk = 0; every row's
+    probabilities sum to 1, hence sum over keys of dv = sum over queries of dout."""
+    L, d, M, N = 90, 8, 16, 6
+    q, k, v = W.random_qkv(1, 2, L, d, 80, std=1.5)
+    dout, _, _ = W.random_qkv(1, 2, L, d, 81)
+    QB, G = -(-L // M), -(-L // N)
+    tiles = W.random_tiles(1, 2, QB, G, 0.3, 82)
+    dq, dk, dv = oracle.backward(q, k, v, dout, W.pack_tiles(tiles), M, N, 0.4)
+    assert np.abs(dk.sum(axis=2)).max() < 1e-10, "sum of dk over keys is not 0"
+    assert np.abs(dv.sum(axis=2) - _f64(dout).sum(axis=2)).max() < 1e-10, "sum of dv != sum of dout"
+
+
+def check_backward_closed_form(oracle):
+    """V = c: every score's gradient vanishes (dP_ij = dout_i . c = D_i), so dq = dk = 0."""
+    L, d, M, N = 60, 8, 16, 4
+    q, k, _ = W.random_qkv(1, 1, L, d, 83)
+    v = torch.full_like(q, -0.75)
+    dout, _, _ = W.random_qkv(1, 1, L, d, 84)
+    QB, G = -(-L // M), -(-L // N)
+    tiles = W.random_tiles(1, 1, QB, G, 0.5, 85)
+    dq, dk, dv = oracle.backward(q, k, v, dout, W.pack_tiles(tiles), M, N, 0.5)
+    assert np.abs(dq).max() < 1e-12 and np.abs(dk).max() < 1e-12, "V=c: dq, dk not 0"
+    assert np.abs(dv).max() > 0.1  # and dv is not trivially zero
+
+
 ALL_CHECKS = [
     check_dense_matches_torch,
     check_brute_force,
@@ -222,4 +278,7 @@ ALL_CHECKS = [
     check_rows_past_end_are_nan,
     check_compaction_brute,
     check_compaction_invariants,
+    check_backward_matches_torch_autograd,
+    check_backward_invariants,
+    check_backward_closed_form,
 ]

@@ -14,6 +14,10 @@ MUTANTS = {
     6: "mask bits read MSB first",
     7: "no division by the normaliser",
     8: "mask ignored",
+    9: "backward: -D term dropped",
+    10: "backward: dk without the scale",
+    11: "backward: unnormalised probabilities",
+    12: "backward: dq accumulates the query",
 }
 
 
