@@ -22,7 +22,7 @@ import torch
 
 from . import _build
 
-__all__ = ["kept_capacity", "compact_mask", "forward", "masked_forward", "masked_forward_noalloc", "attention_from_host",
+__all__ = ["kept_capacity", "compact_mask", "forward", "backward", "masked_forward", "masked_forward_noalloc", "attention_from_host",
            "device_error", "status_string", "num_sms", "FUSED_MAX_WORDS",
            "FgattnError", "LIB_PATH", "DEVERR_BAD_INDEX", "DEVERR_BAD_COUNT", "DEVERR_TIMEOUT"]
 
@@ -57,6 +57,9 @@ def _load() -> ctypes.CDLL:
     lib.fgattn_masked_forward.restype = i32
     lib.fgattn_masked_forward_noalloc.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64, ctypes.c_float, p, p, p]
     lib.fgattn_masked_forward_noalloc.restype = i32
+    lib.fgattn_backward.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float,
+                                    p, p, p, p, p]
+    lib.fgattn_backward.restype = i32
     lib.fgattn_device_error.argtypes = [p, i32, ctypes.POINTER(ctypes.c_uint32)]
     lib.fgattn_device_error.restype = i32
     lib.fgattn_num_sms.argtypes = []
@@ -362,6 +365,53 @@ def masked_forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ma
                                             _stream_ptr(stream))
     _check(st, "fgattn_masked_forward_noalloc")
     return out, lse
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+             lse: torch.Tensor, kept_idx: Optional[torch.Tensor], kept_cnt: Optional[torch.Tensor], M: int, N: int,
+             scale: Optional[float] = None, dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+             dv: Optional[torch.Tensor] = None, delta: Optional[torch.Tensor] = None,
+             stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients of the tile-sparse forward over the same kept lists (None = dense).
+
+    q, k, v, out (the forward's output), dout: contiguous bf16 [B,H,L,d]; lse: the
+    forward's fp32 [B,H,L].  Returns (dq, dk, dv), fp32 [B,H,L,d].  delta (fp32
+    [B,H,L], dO_i . O_i on return) is a workspace, allocated here when not given.
+    dk and dv are sums of float atomics: their last bits depend on the order."""
+    if q.dim() != 4 or any(t.shape != q.shape for t in (k, v, out, dout)):
+        raise ValueError("q, k, v, out, dout must share one [B, H, L, d] shape")
+    B, H, L, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _numel(lse, B * H * L, "lse")
+    if kept_idx is not None and min(L, M, N) >= 1:
+        QB = _geometry(L, M, N)[0]
+        if kept_idx.dim() < 1 or kept_idx.shape[-1] < L:
+            raise ValueError("kept_idx must be [B, H, QB, cap] with cap >= L")
+        _numel(kept_idx, B * H * QB * kept_idx.shape[-1], "kept_idx")
+        _numel(kept_cnt, B * H * QB, "kept_cnt")
+    f32 = (torch.float32,)
+    grads = []
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        if g is None:
+            g = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        _numel(g, B * H * L * d, name)
+        grads.append(g)
+    if delta is None:
+        delta = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _numel(delta, B * H * L, "delta")
+    bf = (torch.bfloat16,)
+    if kept_idx is not None:
+        ip, cp, cap = _dev(kept_idx, "kept_idx", (torch.int32,)), _dev(kept_cnt, "kept_cnt", (torch.int32,)), \
+            kept_idx.shape[-1]
+    else:
+        ip = cp = None
+        cap = L
+    st = _lib.fgattn_backward(_dev(q, "q", bf), _dev(k, "k", bf), _dev(v, "v", bf), _dev(out, "out", bf),
+                              _dev(dout, "dout", bf), _dev(lse, "lse", f32), ip, cp, cap, B, H, L, d, M, N, scale,
+                              _dev(grads[0], "dq", f32), _dev(grads[1], "dk", f32), _dev(grads[2], "dv", f32),
+                              _dev(delta, "delta", f32), _stream_ptr(stream))
+    _check(st, "fgattn_backward")
+    return grads[0], grads[1], grads[2]
 
 
 def device_error(clear: bool = True, stream=None) -> int:

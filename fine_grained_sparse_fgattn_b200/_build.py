@@ -37,7 +37,8 @@ def kernel_hash(kernel: str) -> str:
     """Hash of the sources one kernel is built from (ties a profile to a kernel version)."""
     files = {"fwd": ["attention_fwd.cuh", "mask_row.cuh", "sm100_ptx.cuh"],
              "fwd_qm": ["attention_fwd.cuh", "attention_fwd_qm.cuh", "mask_row.cuh", "sm100_ptx.cuh"],
-             "compact": ["compact_mask.cuh"]}[kernel]
+             "compact": ["compact_mask.cuh"],
+             "bwd": ["attention_fwd.cuh", "attention_bwd.cuh", "mask_row.cuh", "sm100_ptx.cuh"]}[kernel]
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(CSRC, f), "rb") as fh:

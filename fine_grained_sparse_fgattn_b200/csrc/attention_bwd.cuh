@@ -1,0 +1,410 @@
+// Backward pass of tile-sparse softmax attention for sm_100a (tcgen05 + TMEM).
+//
+// The gradients of the forward ("FG-Attn: Leveraging Fine-Grained Sparse
+// Attention in Video Diffusion Models", Abstract: a skipped M x N tile counts as
+// -inf, so its scores have p = 0 and carry no gradient), over the same kept-key
+// lists the forward reads.  With P recomputed from the forward's log-sum-exp,
+//     P^T  = exp(scale * K Q^T - lse)           dP^T = V dO^T
+//     dS^T = P^T o (dP^T - Delta),  Delta_i = dO_i . O_i
+//     dV  += P^T dO      dK += scale * dS^T Q    dQ^T += scale * K^T dS^T
+// per query block (b, h, qb) of MQ rows and each 128-key chunk of its list.
+//
+// Key-major, like the forward's kernel for short query blocks: a thread owns one
+// key of the chunk (TMEM lane), so P^T and dS^T go to TMEM as the A operands of
+// the dV and dK products (M = 128 keys, K = MQ queries), and dS^T also goes to
+// shared memory as the B operand of dQ^T += K^T dS^T (the shape of the
+// forward's O^T += V^T P^T).  dQ^T accumulates in TMEM over the block's chunks
+// and is stored once per block; the chunk's dK and dV rows are added to fp32
+// outputs with vector atomics (one key is kept by many query blocks).
+//
+// One block of 128 threads per SM (persistent, round-robin over query blocks);
+// thread 0 also issues the MMAs.  The K and V rows of the next chunk are loaded
+// with 16-byte cp.async copies (eight or sixteen lanes per row) while the
+// current chunk is computed (two stages).  Every wait is bounded; on a timeout
+// the block sets the device error bit and stops.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "attention_fwd.cuh"
+
+namespace fgattn {
+
+namespace ptx {
+
+// 32 lanes x 8 / 16 consecutive 32-bit TMEM columns from raw words (packed bf16 pairs).
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// Close this thread's outstanding cp.async copies as one group; wait until at most N
+// groups are still in flight.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+}  // namespace ptx
+
+struct BwdParams {
+    const __nv_bfloat16 *q, *k, *v, *dout;  // [B][H][L][D]
+    const float* lse;                        // [B][H][L], natural log (the forward's)
+    const float* delta;                      // [B][H][L], dO_i . O_i
+    const int32_t* kept_idx;                 // [items][cap], or null: every key kept
+    const int32_t* kept_cnt;                 // [items]
+    float *dq, *dk, *dv;                     // fp32 [B][H][L][D]; dk and dv accumulate (zeroed first)
+    int64_t cap, L, QB, items;
+    float scale;       // softmax scale
+    float scale_log2;  // scale * log2(e)
+};
+
+template <int D, int MQ>
+struct BwdCfg {
+    static_assert(D == 64 || D == 128, "head dim");
+    static_assert(MQ == 16 || MQ == 32 || MQ == 64, "query block");
+    static constexpr int KC = 128;                // keys per chunk
+    static constexpr int ROW = D * 2;             // bytes per bf16 row
+    static constexpr int KV_TILE = KC * ROW;      // one chunk of K or V rows
+    static constexpr int Q_TILE = MQ * ROW;       // the block's Q or dO rows
+    static constexpr int P_ROW = (MQ * 2 < 128) ? MQ * 2 : 128;  // bytes per key row of a dS^T panel
+    static constexpr int P_CPR = P_ROW / 16;
+    static constexpr int P_PANEL = KC * P_ROW;
+    static constexpr int P_TILE = KC * MQ * 2;
+    static constexpr int OFF_K = 0;                       // K stages [2]
+    static constexpr int OFF_V = OFF_K + 2 * KV_TILE;     // V stages [2]
+    static constexpr int OFF_Q = OFF_V + 2 * KV_TILE;
+    static constexpr int OFF_DO = OFF_Q + Q_TILE;
+    static constexpr int OFF_DS = OFF_DO + Q_TILE;        // dS^T, MN-major panels
+    static constexpr int OFF_LSE = OFF_DS + P_TILE;       // float [MQ]: lse * log2(e) (+inf past L)
+    static constexpr int OFF_DELTA = OFF_LSE + MQ * 4;    // float [MQ]
+    static constexpr int OFF_BAR = (OFF_DELTA + MQ * 4 + 7) / 8 * 8;  // s_done, g_done, drain
+    static constexpr int OFF_TMEM = OFF_BAR + 3 * 8;
+    static constexpr int OFF_ABORT = OFF_TMEM + 8;
+    static constexpr int BYTES = OFF_ABORT + 8;
+    static constexpr int SMEM_REQUEST = BYTES + 1024;     // + alignment slack
+    static_assert(SMEM_REQUEST <= 227 * 1024, "shared memory");
+    // TMEM columns: S^T, dP^T (MQ fp32 each), P^T and dS^T (MQ / 2 packed bf16 pairs
+    // each), dV and dK (D each, M = 128), dQ^T (MQ columns, M = D)
+    static constexpr uint32_t COL_S = 0, COL_DP = MQ, COL_P = 2 * MQ, COL_DS = COL_P + MQ / 2;
+    static constexpr uint32_t COL_DV = COL_DS + MQ / 2, COL_DK = COL_DV + D, COL_DQ = COL_DK + D;
+    static constexpr uint32_t COLS_USED = COL_DQ + MQ;
+    static constexpr uint32_t TMEM_COLS = COLS_USED <= 128 ? 128 : COLS_USED <= 256 ? 256 : 512;
+    static_assert(COLS_USED <= 512, "TMEM columns");
+};
+
+template <int D, int MQ>
+__global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constant__ BwdParams p) {
+    using C = BwdCfg<D, MQ>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = ptx::smem_u32(smem);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
+    const uint32_t bar_s = sbase + C::OFF_BAR, bar_g = bar_s + 8, bar_drain = bar_s + 16;
+    float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
+    float* s_delta = reinterpret_cast<float*>(smem + C::OFF_DELTA);
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int64_t L = p.L;
+
+    if (warp == 0) {
+        ptx::tmem_alloc(sbase + C::OFF_TMEM, C::TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (t == 0) {
+        ptx::mbar_init(bar_s, 1);
+        ptx::mbar_init(bar_g, 1);
+        ptx::mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + C::OFF_TMEM);
+
+    // Rows r0 .. r0+nrows of a K-major 128B-swizzled tile (64-column panels of prow
+    // rows) from base[key_of(r)] (zero-filled where key_of returns -1): one 16-byte
+    // piece per lane, PPR lanes per row.
+    constexpr int PPR = D / 8;
+    constexpr int RPI = 32 / PPR;  // rows per warp instruction
+    auto load_rows = [&](uint32_t dst, int prow, const __nv_bfloat16* base, int r0, int nrows, auto key_of) {
+        for (int i = 0; i < nrows / RPI; ++i) {
+            const int r = r0 + i * RPI + lane / PPR;
+            const int pc = lane % PPR;
+            const int64_t key = key_of(r);
+            const __nv_bfloat16* src = base + (key >= 0 ? key : 0) * D + pc * 8;
+            ptx::cp_async_16(dst + (uint32_t)(pc / 8) * (uint32_t)(prow * 128) + swz((uint32_t)r, (uint32_t)(pc % 8), 128u),
+                             src, key >= 0 ? 16u : 0u);
+        }
+    };
+
+    uint32_t ph_s = 0, ph_g = 0;  // phases of the two MMA barriers
+    bool failed = false;
+    int64_t gcount = 0;  // chunks this block has processed (stage parity)
+    for (int64_t item = blockIdx.x; item < p.items && !failed; item += gridDim.x) {
+        const int64_t bh = item / p.QB, qb = item - bh * p.QB;
+        int64_t cnt = L;
+        const int32_t* lst = nullptr;
+        if (p.kept_idx != nullptr) {
+            cnt = p.kept_cnt[item];
+            if (cnt < 1 || cnt > p.cap) {
+                if (t == 0) atomicOr(&g_device_error, kErrBadCount);
+                cnt = cnt < 1 ? 1 : p.cap;
+            }
+            lst = p.kept_idx + item * p.cap;
+        }
+        const int64_t nch = (cnt + 127) / 128;
+        const __nv_bfloat16* kb = p.k + bh * L * D;
+        const __nv_bfloat16* vb = p.v + bh * L * D;
+        const int64_t row0 = qb * MQ;
+        // key at list position j (checked), or 0 past the list
+        auto key_at = [&](int64_t j) -> int64_t {
+            if (j >= cnt) return 0;
+            if (lst == nullptr) return j;
+            int32_t x = __ldg(lst + j);
+            if (x < 0 || (int64_t)x >= L) {
+                atomicOr(&g_device_error, kErrBadIndex);
+                x = 0;
+            }
+            return x;
+        };
+        // ---- the block's Q and dO rows (zero past L), lse in log2 units and Delta
+        {
+            auto qrow = [&](int r) -> int64_t { return row0 + r < L ? row0 + r : -1; };
+            load_rows(sbase + C::OFF_Q, MQ, p.q + bh * L * D, warp * (MQ / 4), MQ / 4, qrow);
+            load_rows(sbase + C::OFF_DO, MQ, p.dout + bh * L * D, warp * (MQ / 4), MQ / 4, qrow);
+            ptx::cp_async_commit();
+            if (t < MQ) {
+                const bool in = row0 + t < L;
+                s_lse[t] = in ? p.lse[bh * L + row0 + t] * 1.4426950408889634f : INFINITY;
+                s_delta[t] = in ? p.delta[bh * L + row0 + t] : 0.f;
+            }
+        }
+        // K and V rows of chunk c into stage (gcount + c) & 1
+        auto issue_chunk = [&](int64_t c) {
+            const uint32_t st = (uint32_t)((gcount + c) & 1);
+            auto key_of = [&](int r) -> int64_t { return key_at(c * 128 + r); };
+            load_rows(sbase + C::OFF_K + st * C::KV_TILE, 128, kb, warp * 32, 32, key_of);
+            load_rows(sbase + C::OFF_V + st * C::KV_TILE, 128, vb, warp * 32, 32, key_of);
+            ptx::cp_async_commit();
+        };
+        issue_chunk(0);
+        for (int64_t c = 0; c < nch; ++c) {
+            const uint32_t st = (uint32_t)((gcount + c) & 1);
+            if (c + 1 < nch) {
+                issue_chunk(c + 1);
+                ptx::cp_async_wait_group<1>();  // all but the newest group have landed
+            } else {
+                ptx::cp_async_wait_group<0>();
+            }
+            ptx::fence_proxy_async_smem();  // this thread's copies -> visible to the tensor core
+            ptx::tc_fence_before();
+            __syncthreads();
+            ptx::tc_fence_after();
+            const uint32_t kst = sbase + C::OFF_K + st * C::KV_TILE;
+            const uint32_t vst = sbase + C::OFF_V + st * C::KV_TILE;
+            // ---- S^T = K Q^T and dP^T = V dO^T (K-major operands, M = 128 keys, N = MQ)
+            if (t == 0) {
+                constexpr uint32_t IDESC = umma_idesc_bf16(128, MQ, false, false);
+                constexpr uint32_t HI = umma_desc_hi(1024u, 2u);
+                const uint32_t klo = umma_desc_lo(kst, 16u), vlo = umma_desc_lo(vst, 16u);
+                const uint32_t qlo = umma_desc_lo(sbase + C::OFF_Q, 16u);
+                const uint32_t olo = umma_desc_lo(sbase + C::OFF_DO, 16u);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t aoff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
+                    const uint32_t boff = (uint32_t)(kk / 4) * (MQ * 128) + (uint32_t)(kk % 4) * 32u;
+                    ptx::mma_bf16_ss(tmem + C::COL_S, umma_desc_join(klo + (aoff >> 4), HI),
+                                     umma_desc_join(qlo + (boff >> 4), HI), IDESC, kk > 0 ? 1u : 0u);
+                    ptx::mma_bf16_ss(tmem + C::COL_DP, umma_desc_join(vlo + (aoff >> 4), HI),
+                                     umma_desc_join(olo + (boff >> 4), HI), IDESC, kk > 0 ? 1u : 0u);
+                }
+                ptx::mma_commit(bar_s);
+            }
+            if (!bounded_wait(bar_s, ph_s, abort_flag)) failed = true;
+            ph_s ^= 1u;
+            ptx::tc_fence_after();
+            // ---- P^T and dS^T of this thread's key, up to 32 query columns at a time
+            const bool valid = c * 128 + t < cnt;
+            constexpr int QW = MQ < 32 ? MQ : 32;
+#pragma unroll 1
+            for (int q0 = 0; q0 < MQ; q0 += QW) {
+                float sv[QW], dp[QW];
+                if constexpr (QW == 32) {
+                    ptx::tmem_ld32(tmem + C::COL_S + (uint32_t)q0 + lane_base, sv);
+                    ptx::tmem_ld32(tmem + C::COL_DP + (uint32_t)q0 + lane_base, dp);
+                } else {
+                    ptx::tmem_ld16(tmem + C::COL_S + (uint32_t)q0 + lane_base, sv);
+                    ptx::tmem_ld16(tmem + C::COL_DP + (uint32_t)q0 + lane_base, dp);
+                }
+                ptx::tmem_wait_ld();
+                uint32_t pp[QW / 2], dd[QW / 2];
+#pragma unroll
+                for (int j = 0; j < QW; j += 2) {
+                    float pr[2], ds[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int q = q0 + j + e;
+                        pr[e] = valid ? ptx::ex2(fmaf(sv[j + e], p.scale_log2, -s_lse[q])) : 0.f;
+                        ds[e] = pr[e] * (dp[j + e] - s_delta[q]);
+                    }
+                    __nv_bfloat162 hp = __floats2bfloat162_rn(pr[0], pr[1]);
+                    __nv_bfloat162 hd = __floats2bfloat162_rn(ds[0], ds[1]);
+                    pp[j / 2] = *reinterpret_cast<uint32_t*>(&hp);
+                    dd[j / 2] = *reinterpret_cast<uint32_t*>(&hd);
+                }
+                // P^T and dS^T rows of this key into TMEM (A operands: two queries per column)
+                if constexpr (QW == 32) {
+                    ptx::tmem_st16u(tmem + C::COL_P + (uint32_t)(q0 / 2) + lane_base, pp);
+                    ptx::tmem_st16u(tmem + C::COL_DS + (uint32_t)(q0 / 2) + lane_base, dd);
+                } else {
+                    ptx::tmem_st8u(tmem + C::COL_P + (uint32_t)(q0 / 2) + lane_base, pp);
+                    ptx::tmem_st8u(tmem + C::COL_DS + (uint32_t)(q0 / 2) + lane_base, dd);
+                }
+                // the dS^T row into shared memory (B operand of dQ^T: MN-major, queries contiguous)
+#pragma unroll
+                for (int j = 0; j < QW; j += 8) {
+                    const int chunk = (q0 + j) / 8;  // 16-byte chunk = 8 queries
+                    const int panel = chunk / C::P_CPR;
+                    const uint32_t addr = sbase + C::OFF_DS + (uint32_t)panel * C::P_PANEL +
+                                          swz((uint32_t)t, (uint32_t)(chunk % C::P_CPR), (uint32_t)C::P_ROW);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dd[j / 2]),
+                                 "r"(dd[j / 2 + 1]), "r"(dd[j / 2 + 2]), "r"(dd[j / 2 + 3])
+                                 : "memory");
+                }
+            }
+            ptx::tmem_wait_st();
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            __syncthreads();
+            ptx::tc_fence_after();
+            // ---- dV = P^T dO and dK = dS^T Q (A in TMEM; B = the Q / dO tiles read
+            //      MN-major), dQ^T += K^T dS^T (A = the K stage read MN-major; B = dS^T)
+            if (t == 0) {
+                constexpr uint32_t IDESC_KV = umma_idesc_bf16(128, D, false, true);
+                constexpr uint32_t IDESC_Q = umma_idesc_bf16(D, MQ, true, true);
+                constexpr uint32_t HI_T = umma_desc_hi(1024u, 2u);
+                constexpr uint32_t P_LAYOUT = (C::P_ROW == 128) ? 2u : (C::P_ROW == 64) ? 4u : 6u;
+                constexpr uint32_t HI_DS = umma_desc_hi(8u * C::P_ROW, P_LAYOUT);
+                const uint32_t olo = umma_desc_lo(sbase + C::OFF_DO, (uint32_t)(MQ * 128));
+                const uint32_t qlo = umma_desc_lo(sbase + C::OFF_Q, (uint32_t)(MQ * 128));
+                const uint32_t klo = umma_desc_lo(kst, 128u * 128u);
+                const uint32_t dlo = umma_desc_lo(sbase + C::OFF_DS, (uint32_t)C::P_PANEL);
+#pragma unroll
+                for (int kk = 0; kk < MQ / 16; ++kk) {  // over the block's queries
+                    ptx::mma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_P + (uint32_t)kk * 8u,
+                                     umma_desc_join(olo + (uint32_t)(kk * 2048 >> 4), HI_T), IDESC_KV,
+                                     kk > 0 ? 1u : 0u);
+                    ptx::mma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DS + (uint32_t)kk * 8u,
+                                     umma_desc_join(qlo + (uint32_t)(kk * 2048 >> 4), HI_T), IDESC_KV,
+                                     kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // over the chunk's keys
+                    ptx::mma_bf16_ss(tmem + C::COL_DQ, umma_desc_join(klo + (uint32_t)(kk * 2048 >> 4), HI_T),
+                                     umma_desc_join(dlo + (uint32_t)(kk * 16 * C::P_ROW >> 4), HI_DS), IDESC_Q,
+                                     (c > 0 || kk > 0) ? 1u : 0u);
+                ptx::mma_commit(bar_g);
+            }
+            if (!bounded_wait(bar_g, ph_g, abort_flag)) failed = true;
+            ph_g ^= 1u;
+            ptx::tc_fence_after();
+            // ---- this key's dV and dK rows into the fp32 outputs (every lane reads TMEM;
+            //      only lanes of list keys store)
+            {
+                const int64_t key = valid ? key_at(c * 128 + t) : -1;
+                float* dvr = p.dv + (bh * L + (key >= 0 ? key : 0)) * D;
+                float* dkr = p.dk + (bh * L + (key >= 0 ? key : 0)) * D;
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    float a[32], b[32];
+                    ptx::tmem_ld32(tmem + C::COL_DV + (uint32_t)c0 + lane_base, a);
+                    ptx::tmem_ld32(tmem + C::COL_DK + (uint32_t)c0 + lane_base, b);
+                    ptx::tmem_wait_ld();
+                    if (key >= 0) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            atomicAdd(reinterpret_cast<float4*>(dvr + c0 + e),
+                                      make_float4(a[e], a[e + 1], a[e + 2], a[e + 3]));
+                            atomicAdd(reinterpret_cast<float4*>(dkr + c0 + e),
+                                      make_float4(p.scale * b[e], p.scale * b[e + 1], p.scale * b[e + 2],
+                                                  p.scale * b[e + 3]));
+                        }
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncthreads();  // TMEM dV / dK, dS^T and the K stage are free for the next chunk
+            ptx::tc_fence_after();
+        }
+        gcount += nch;
+        // ---- dQ rows of the block: dQ^T has D lanes x MQ columns (at D = 64 the M = 64
+        //      accumulator holds row 16 * warp + lane in lanes 0..15 of each warp)
+        const int dt = (D == 128) ? t : ((lane < 16) ? warp * 16 + lane : -1);
+#pragma unroll 1
+        for (int q0 = 0; q0 < MQ; q0 += 8) {
+            float o[8];
+            ptx::tmem_ld8(tmem + C::COL_DQ + (uint32_t)q0 + lane_base, o);
+            ptx::tmem_wait_ld();
+            if (dt >= 0) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int64_t row = row0 + q0 + j;
+                    if (row < L) p.dq[(bh * L + row) * D + dt] = p.scale * o[j];
+                }
+            }
+        }
+        ptx::tc_fence_before();
+        // dQ^T read before the next block's first product overwrites it; leave together
+        failed = __syncthreads_or(failed);
+        ptx::tc_fence_after();
+    }
+    // drain: every MMA issued has completed before TMEM is freed
+    if (t == 0) {
+        ptx::mma_commit(bar_drain);
+        bounded_wait(bar_drain, 0u, abort_flag, /*honour_abort=*/false);
+    }
+    ptx::cp_async_wait_all();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 0) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// Delta_i = dO_i . O_i in fp32, one warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) fgattn_bwd_delta_kernel(const __nv_bfloat16* __restrict__ out,
+                                                               const __nv_bfloat16* __restrict__ dout,
+                                                               float* __restrict__ delta, int64_t rows) {
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float acc = 0.f;
+#pragma unroll
+    for (int e = lane * 2; e < D; e += 64) {
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(out + row * D + e);
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(dout + row * D + e);
+        acc = fmaf(__bfloat162float(a.x), __bfloat162float(b.x), acc);
+        acc = fmaf(__bfloat162float(a.y), __bfloat162float(b.y), acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) delta[row] = acc;
+}
+
+}  // namespace fgattn

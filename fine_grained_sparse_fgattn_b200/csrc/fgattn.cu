@@ -1,8 +1,8 @@
 // C ABI of the tile-sparse attention library (declared in include/fgattn.h).
 // Host side only: argument validation, launch configuration, device error
 // word, the host-to-host copy pipeline and the allocation-free entry point.
-// The kernels are in compact_mask.cuh, attention_fwd.cuh (key-major) and
-// attention_fwd_qm.cuh (query-major).
+// The kernels are in compact_mask.cuh, attention_fwd.cuh (key-major),
+// attention_fwd_qm.cuh (query-major) and attention_bwd.cuh (gradients).
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "fgattn.h"
+#include "attention_bwd.cuh"
 #include "attention_fwd.cuh"
 #include "attention_fwd_qm.cuh"
 #include "compact_mask.cuh"
@@ -424,6 +425,96 @@ fgattn_status fgattn_masked_forward(const void* q, const void* k, const void* v,
     if (W > fgattn::kFusedMaxWords) return FGATTN_ERR_UNSUPPORTED;
     const Strides c = {{H * L * d, L * d, d}};  // contiguous [B][H][L][d]
     return forward_impl(q, c, k, c, v, c, nullptr, nullptr, L, B, H, L, d, M, N, scale, out, c, lse, stream, mask);
+}
+
+}  // extern "C"
+
+namespace {
+
+template <int D, int MQ>
+fgattn_status launch_bwd(const fgattn::BwdParams& prm, cudaStream_t s) {
+    using C = fgattn::BwdCfg<D, MQ>;
+    auto kernel = fgattn::fgattn_bwd_kernel<D, MQ>;
+    // one block per SM: the block allocates up to all of the SM's TMEM columns
+    const int smem = C::SMEM_REQUEST > 120 * 1024 ? C::SMEM_REQUEST : 120 * 1024;
+    static bool configured[kMaxConfigDevices] = {};
+    int cdev = 0;
+    if (cudaGetDevice(&cdev) != cudaSuccess || cdev < 0 || cdev >= kMaxConfigDevices) return FGATTN_ERR_CUDA;
+    if (!configured[cdev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return FGATTN_ERR_CUDA;
+        configured[cdev] = true;
+    }
+    const int sms = current_sms();
+    if (sms <= 0) return FGATTN_ERR_CUDA;
+    const int64_t grid = prm.items < sms ? prm.items : sms;
+    kernel<<<(unsigned)grid, 128, smem, s>>>(prm);
+    return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
+}
+
+template <int D>
+fgattn_status launch_bwd_m(const fgattn::BwdParams& prm, int64_t M, cudaStream_t s) {
+    switch (M) {
+        case 16: return launch_bwd<D, 16>(prm, s);
+        case 32: return launch_bwd<D, 32>(prm, s);
+        default: return launch_bwd<D, 64>(prm, s);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                              const float* lse, const int32_t* kept_idx, const int32_t* kept_cnt, int64_t cap,
+                              int64_t B, int64_t H, int64_t L, int64_t d, int64_t M, int64_t N, float scale,
+                              float* dq, float* dk, float* dv, float* delta, fgattn_stream_t stream) {
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta) return FGATTN_ERR_INVALID_ARG;
+    if (kept_idx && !kept_cnt) return FGATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || L < 1 || M < 1 || N < 1 || d < 1) return FGATTN_ERR_INVALID_ARG;
+    if (L > INT32_MAX || B > INT32_MAX || H > INT32_MAX) return FGATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return FGATTN_ERR_INVALID_ARG;
+    for (const void* ptr : {q, k, v, out, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+        if (!aligned16(ptr)) return FGATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(delta) & 3u) ||
+        (kept_idx && (reinterpret_cast<uintptr_t>(kept_idx) & 3u)))
+        return FGATTN_ERR_INVALID_ARG;
+    if (kept_idx && (cap < L || (cap & 3))) return FGATTN_ERR_CAPACITY;
+    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (M != 16 && M != 32 && M != 64) return FGATTN_ERR_UNSUPPORTED;
+    if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t rows = B * H * L;
+    const size_t grad_bytes = (size_t)rows * (size_t)d * sizeof(float);
+    if (cudaMemsetAsync(dk, 0, grad_bytes, s) != cudaSuccess) return FGATTN_ERR_CUDA;
+    if (cudaMemsetAsync(dv, 0, grad_bytes, s) != cudaSuccess) return FGATTN_ERR_CUDA;
+    const auto* ob = static_cast<const __nv_bfloat16*>(out);
+    const auto* gb = static_cast<const __nv_bfloat16*>(dout);
+    const unsigned dblocks = (unsigned)((rows + 7) / 8);
+    if (d == 128)
+        fgattn::fgattn_bwd_delta_kernel<128><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
+    else
+        fgattn::fgattn_bwd_delta_kernel<64><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
+    if (cudaPeekAtLastError() != cudaSuccess) return FGATTN_ERR_CUDA;
+    fgattn::BwdParams prm;
+    prm.q = static_cast<const __nv_bfloat16*>(q);
+    prm.k = static_cast<const __nv_bfloat16*>(k);
+    prm.v = static_cast<const __nv_bfloat16*>(v);
+    prm.dout = gb;
+    prm.lse = lse;
+    prm.delta = delta;
+    prm.kept_idx = kept_idx;
+    prm.kept_cnt = kept_cnt;
+    prm.dq = dq;
+    prm.dk = dk;
+    prm.dv = dv;
+    prm.cap = kept_idx ? cap : L;
+    prm.L = L;
+    prm.QB = (L + M - 1) / M;
+    prm.items = B * H * prm.QB;
+    prm.scale = scale;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    return d == 128 ? launch_bwd_m<128>(prm, M, s) : launch_bwd_m<64>(prm, M, s);
 }
 
 fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* bits) {

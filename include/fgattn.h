@@ -158,6 +158,36 @@ fgattn_status fgattn_masked_forward(const void* q, const void* k, const void* v,
                                     float* lse, fgattn_stream_t stream);
 
 /*
+ * Gradients of the tile-sparse forward ("FG-Attn ...", Abstract: a skipped
+ * tile's scores are -inf, so p = 0 there and they carry no gradient; the page
+ * gives only the forward, and this is its derivative).  Over the kept keys j
+ * of each query row i, with p_ij = exp(scale * q_i . k_j - lse_i) recomputed
+ * and g_i = dout_i:
+ *   dp_ij = g_i . v_j,  delta_i = g_i . out_i,  ds_ij = p_ij (dp_ij - delta_i),
+ *   dq_i = scale * sum_j ds_ij k_j,  dk_j = scale * sum_i ds_ij q_i,
+ *   dv_j = sum_i p_ij g_i.
+ *   q, k, v, out, dout  in   device bf16 [B][H][L][d] (out and lse as the
+ *                            forward wrote them for the same lists and scale)
+ *   lse                 in   device fp32 [B][H][L]
+ *   kept_idx, kept_cnt  in   as for fgattn_forward (NULL kept_idx = dense)
+ *   dq, dk, dv          out  device fp32 [B][H][L][d], 16-byte aligned; every
+ *                            element is written (rows of keys that no query
+ *                            block keeps get zeros)
+ *   delta               out  device fp32 [B][H][L]: workspace owned by the
+ *                            caller; holds delta_i on return
+ * Supported: d in {64, 128}, M in {16, 32, 64}, any N >= 1, any L >= 1.
+ * P and ds are rounded to bf16 for the tensor-core products; accumulation in
+ * fp32.  dk and dv are accumulated with float atomics (many query blocks keep
+ * one key), so their last bits depend on the order the blocks run in; dq is
+ * deterministic.  Errors: INVALID_ARG, UNSUPPORTED, CAPACITY, CUDA; device-side
+ * problems as for fgattn_forward.
+ */
+fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                              const float* lse, const int32_t* kept_idx, const int32_t* kept_cnt, int64_t cap,
+                              int64_t B, int64_t H, int64_t L, int64_t d, int64_t M, int64_t N, float scale,
+                              float* dq, float* dk, float* dv, float* delta, fgattn_stream_t stream);
+
+/*
  * Synchronise `stream`, then report (and, if clear != 0, reset) the device
  * error bits (FGATTN_DEVERR_*) recorded on the current device since the last
  * clear.  *bits may be NULL.  Returns DEVICE if any bit is set, CUDA if the

@@ -135,6 +135,51 @@ def test_masked_forward_rejects(kw, status):
     assert _mfwd(**kw) == status
 
 
+def _bwd(**kw):
+    a = dict(q=P, k=P, v=P, out=P, dout=P, lse=P, idx=P, cnt=P, cap=64, B=1, H=1, L=64, d=128, M=64, N=16,
+             scale=0.1, dq=P, dk=P, dv=P, delta=P)
+    a.update(kw)
+    return F._lib.fgattn_backward(a["q"], a["k"], a["v"], a["out"], a["dout"], a["lse"], a["idx"], a["cnt"],
+                                  a["cap"], a["B"], a["H"], a["L"], a["d"], a["M"], a["N"], a["scale"], a["dq"],
+                                  a["dk"], a["dv"], a["delta"], None)
+
+
+def test_header_declares_backward():
+    assert "fgattn_backward" in declared_functions()
+
+
+@no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), F.ERR_INVALID_ARG),
+    (dict(out=None), F.ERR_INVALID_ARG),
+    (dict(dout=None), F.ERR_INVALID_ARG),
+    (dict(lse=None), F.ERR_INVALID_ARG),
+    (dict(dq=None), F.ERR_INVALID_ARG),
+    (dict(dk=None), F.ERR_INVALID_ARG),
+    (dict(dv=None), F.ERR_INVALID_ARG),
+    (dict(delta=None), F.ERR_INVALID_ARG),
+    (dict(cnt=None), F.ERR_INVALID_ARG),
+    (dict(L=0), F.ERR_INVALID_ARG),
+    (dict(N=0), F.ERR_INVALID_ARG),
+    (dict(scale=float("inf")), F.ERR_INVALID_ARG),
+    (dict(dout=P + 8), F.ERR_INVALID_ARG),
+    (dict(dk=P + 4), F.ERR_INVALID_ARG),
+    (dict(delta=P + 2), F.ERR_INVALID_ARG),
+    (dict(cap=63), F.ERR_CAPACITY),
+    (dict(d=96), F.ERR_UNSUPPORTED),
+    (dict(d=80), F.ERR_UNSUPPORTED),
+    (dict(M=128), F.ERR_UNSUPPORTED),
+    (dict(M=48), F.ERR_UNSUPPORTED),
+])
+def test_backward_rejects(kw, status):
+    assert _bwd(**kw) == status
+
+
+@no_gpu
+def test_backward_valid_call_without_gpu_reports_cuda_error():
+    assert _bwd() == F.ERR_CUDA
+
+
 @no_gpu
 def test_valid_call_without_gpu_reports_cuda_error():
     # All arguments valid, so the launch is attempted; with no device it fails cleanly.

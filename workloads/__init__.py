@@ -290,3 +290,9 @@ def random_qkv(B: int, H: int, L: int, d: int, seed: int, std: float = 1.0):
     k = (torch.randn((B, H, L, d), generator=g) * std).to(torch.bfloat16)
     v = torch.randn((B, H, L, d), generator=g).to(torch.bfloat16)
     return q, k, v
+
+
+def random_grad(B: int, H: int, L: int, d: int, seed: int, std: float = 1.0) -> torch.Tensor:
+    """iid N(0, std^2) bf16 upstream gradient dO [B, H, L, d] (backward cases)."""
+    g = _torch_gen(seed, "fuzzgrad", B, H, L, d)
+    return (torch.randn((B, H, L, d), generator=g) * std).to(torch.bfloat16)
