@@ -257,6 +257,131 @@ def profile_key(w, args):
 
 
 # ---------------------------------------------------------------------------
+# backward mode: gradients of one attention call over the forward's kept lists
+# ---------------------------------------------------------------------------
+BWD_METRIC = "effective TFLOP/s of the backward (unskipped; 10 d FLOP per kept score) & ms per call"
+
+
+def run_backward(args, w, F):
+    """One step = fgattn_backward on resident q, k, v, out, dO, lse and kept lists
+    (the delta pass, zeroing dk/dv and the gradient kernel).  The forward and the
+    compaction that produce its inputs run once, before timing."""
+    rank, world, dist = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    heads = head_shard(w.H, rank)
+    B, H, L, d, M, N = w.B, w.H, w.L, w.d, w.M, w.N
+    QB = w.QB
+    q_h, k_h, v_h = W.make_qkv(w, args.seed, heads=heads)
+    g_h = W.random_grad(B, H, L, d, seed=args.seed + 17)
+    mask_h = W.make_mask(w, args.seed, heads=heads)
+    q, k, v, g = (t.to(dev) for t in (q_h, k_h, v_h, g_h))
+    mask = torch.from_numpy(mask_h.view(np.int32)).to(dev)
+    cap = F.kept_capacity(L)
+    kept_idx = torch.empty((B, H, QB, cap), dtype=torch.int32, device=dev)
+    kept_cnt = torch.empty((B, H, QB), dtype=torch.int32, device=dev)
+    F.compact_mask(mask, B, H, L, M, N, kept_idx=kept_idx, kept_cnt=kept_cnt, cap=cap)
+    out, lse = F.forward(q, k, v, kept_idx, kept_cnt, M, N, w.scale)
+    dq, dk, dv = (torch.empty((B, H, L, d), dtype=torch.float32, device=dev) for _ in range(3))
+    delta = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        F.backward(q, k, v, out, g, lse, kept_idx, kept_cnt, M, N, w.scale, dq=dq, dk=dk, dv=dv, delta=delta)
+
+    step()
+    assert F.device_error() == 0, "device error on the first step"
+    rows = torch.clamp(L - torch.arange(QB, device=dev) * M, max=M).to(torch.float64)
+    kept_scores = float((kept_cnt.to(torch.float64) * rows).sum().item())
+    flops_per_step = 10.0 * d * kept_scores
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, out, g, kept_idx))
+    flush = in_bytes < 2 * L2_BYTES
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
+    for _ in range(args.warmup):
+        if flush:
+            flush_buf.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(dist)
+    torch.cuda.synchronize()
+    with sampler:
+        t_start.record(stream)
+        for i in range(args.steps):
+            if flush:
+                flush_buf.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(dist)
+    bwd_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev), dist)
+    total_ms = reduce_max(t_start.elapsed_time(t_end), dist)
+    clocks = sampler.summary()
+    assert F.device_error() == 0, "device error in the timed region"
+    ms_per_step = bwd_ms if flush else total_ms / args.steps
+    value = job_throughput(world, flops_per_step, ms_per_step)
+
+    # ---- end to end: pinned host inputs -> compaction + backward -> gradients on the host
+    pins = [t.pin_memory() for t in (q_h, k_h, v_h, g_h)]
+    out_p, lse_p = out.cpu().pin_memory(), lse.cpu().pin_memory()
+    mask_p = torch.from_numpy(mask_h.view(np.int32)).pin_memory()
+    grads_h = [torch.empty((B, H, L, d), dtype=torch.float32).pin_memory() for _ in range(3)]
+    out_d, lse_d = torch.empty_like(out), torch.empty_like(lse)
+    h2d = sum(t.numel() * t.element_size() for t in pins + [out_p, lse_p, mask_p])
+    d2h = sum(t.numel() * t.element_size() for t in grads_h)
+
+    def e2e_step():
+        for dst, src in zip((q, k, v, g, out_d, lse_d, mask), pins + [out_p, lse_p, mask_p]):
+            dst.copy_(src, non_blocking=True)
+        F.compact_mask(mask, B, H, L, M, N, kept_idx=kept_idx, kept_cnt=kept_cnt, cap=cap)
+        F.backward(q, k, v, out_d, g, lse_d, kept_idx, kept_cnt, M, N, w.scale, dq=dq, dk=dk, dv=dv, delta=delta)
+        for dst, src in zip(grads_h, (dq, dk, dv)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(dist)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dist) / args.e2e_steps
+    assert F.device_error() == 0, "device error in the end-to-end steps"
+
+    peaks, peak_kind = load_peaks()
+    achieved = flops_per_step / (bwd_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "peak_kind": f"{peak_kind} bf16 burst", "kernel": f"fgattn_bwd_kernel<{d},{M}>",
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "flops_per_launch": flops_per_step,
+                "timed": "delta pass + dk/dv zeroing + gradient kernel (one fgattn_backward call)"}
+    if rank == 0:
+        cfg = cfg_dict(w, args, flush)
+        cfg["path"] = "tile-sparse backward (fgattn_backward over the forward's kept lists)"
+        line = {
+            "metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "backward_ms": bwd_ms, "achieved_sparsity": 1.0 - kept_scores / (B * H * float(L) * L),
+            "roofline": roofline, "cpu_baseline": None,
+            "e2e": {"value": job_throughput(world, flops_per_step, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "mode": "copy in, compaction + backward, copy dq/dk/dv out (serial)"},
+            "gpu_launches": 2 * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -280,6 +405,8 @@ def main():
     ap.add_argument("--fused", action="store_true",
                     help="one kernel per step: the forward reads the mask in place of kept lists "
                          "(fgattn_masked_forward; compaction fused into the forward)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the gradients (fgattn_backward) of the workload's attention call instead")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.get(args.workload)
@@ -294,6 +421,8 @@ def main():
 
     import fine_grained_sparse_fgattn_b200 as F  # fails loudly without the CUDA library
 
+    if args.backward:
+        return run_backward(args, w, F)
     rank, world, dist = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
     heads = head_shard(w.H, rank)

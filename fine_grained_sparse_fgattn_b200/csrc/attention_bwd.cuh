@@ -14,14 +14,20 @@
 // the dV and dK products (M = 128 keys, K = MQ queries), and dS^T also goes to
 // shared memory as the B operand of dQ^T += K^T dS^T (the shape of the
 // forward's O^T += V^T P^T).  dQ^T accumulates in TMEM over the block's chunks
-// and is stored once per block; the chunk's dK and dV rows are added to fp32
-// outputs with vector atomics (one key is kept by many query blocks).
+// and is stored once per block.  A key is kept by many query blocks, so the
+// chunk's dK and dV rows are ADDED to fp32 outputs, by the TMA unit: each warp
+// stages its 32 rows in shared memory, 32 columns at a time, and a run of 16
+// consecutive keys (what a list of 16-key groups is made of) goes out as one
+// 16 x 32 box reduction; any other row goes out as one 128-byte bulk reduction.
+// The adds happen in L2, with no per-thread atomics.
 //
 // One block of 128 threads per SM (persistent, round-robin over query blocks);
-// thread 0 also issues the MMAs.  The K and V rows of the next chunk are loaded
-// with 16-byte cp.async copies (eight or sixteen lanes per row) while the
-// current chunk is computed (two stages).  Every wait is bounded; on a timeout
-// the block sets the device error bit and stops.
+// thread 0 also issues the MMAs.  Per chunk c: softmax(c); then the dV/dK/dQ
+// products of c and, behind them, the score products of c+1, so that the
+// tensor core computes S(c+1) while the threads write out dK/dV of c.  The K and
+// V rows of chunk c+2 are loaded with 16-byte cp.async copies into the stage of
+// chunk c once its products are done (two stages).  Every wait is bounded; on a
+// timeout the block sets the device error bit and stops.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -59,9 +65,32 @@ __device__ __forceinline__ void cp_async_wait_group() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// TMA reduction: add the fp32 box at shared address src into the tensor at
+// coordinates {x, y, z} (the tensor map fixes the box and the swizzle).
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int32_t x, int32_t y, int32_t z) {
+    asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y), "r"(z), "r"(src)
+                 : "memory");
+}
+
+// Add `bytes` (a multiple of 16) contiguous fp32 values at shared address src to dst.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst), "r"(src),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every bulk group of this thread has finished reading its shared-memory source
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every bulk group of this thread has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 }  // namespace ptx
 
-struct BwdParams {
+struct alignas(64) BwdParams {
+    CUtensorMap tmap_dk, tmap_dv;            // fp32 {D, L, B*H}, box {32, 16, 1}, 128B swizzle
     const __nv_bfloat16 *q, *k, *v, *dout;  // [B][H][L][D]
     const float* lse;                        // [B][H][L], natural log (the forward's)
     const float* delta;                      // [B][H][L], dO_i . O_i
@@ -85,12 +114,14 @@ struct BwdCfg {
     static constexpr int P_CPR = P_ROW / 16;
     static constexpr int P_PANEL = KC * P_ROW;
     static constexpr int P_TILE = KC * MQ * 2;
+    static constexpr int STG = KC * 128;          // one staged 32-column slice of dV or dK (fp32)
     static constexpr int OFF_K = 0;                       // K stages [2]
     static constexpr int OFF_V = OFF_K + 2 * KV_TILE;     // V stages [2]
     static constexpr int OFF_Q = OFF_V + 2 * KV_TILE;
     static constexpr int OFF_DO = OFF_Q + Q_TILE;
     static constexpr int OFF_DS = OFF_DO + Q_TILE;        // dS^T, MN-major panels
-    static constexpr int OFF_LSE = OFF_DS + P_TILE;       // float [MQ]: lse * log2(e) (+inf past L)
+    static constexpr int OFF_STG = OFF_DS + P_TILE;       // dV slice, dK slice: [8 runs][16 rows][128 B]
+    static constexpr int OFF_LSE = OFF_STG + 2 * STG;     // float [MQ]: lse * log2(e) (+inf past L)
     static constexpr int OFF_DELTA = OFF_LSE + MQ * 4;    // float [MQ]
     static constexpr int OFF_BAR = (OFF_DELTA + MQ * 4 + 7) / 8 * 8;  // s_done, g_done, drain
     static constexpr int OFF_TMEM = OFF_BAR + 3 * 8;
@@ -98,6 +129,7 @@ struct BwdCfg {
     static constexpr int BYTES = OFF_ABORT + 8;
     static constexpr int SMEM_REQUEST = BYTES + 1024;     // + alignment slack
     static_assert(SMEM_REQUEST <= 227 * 1024, "shared memory");
+    static_assert(OFF_STG % 1024 == 0, "staged boxes need 1024-byte aligned 128B-swizzle atoms");
     // TMEM columns: S^T, dP^T (MQ fp32 each), P^T and dS^T (MQ / 2 packed bf16 pairs
     // each), dV and dK (D each, M = 128), dQ^T (MQ columns, M = D)
     static constexpr uint32_t COL_S = 0, COL_DP = MQ, COL_P = 2 * MQ, COL_DS = COL_P + MQ / 2;
@@ -153,9 +185,58 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
         }
     };
 
+    // S^T = K Q^T and dP^T = V dO^T of the chunk in stage st (K-major operands,
+    // M = 128 keys, N = MQ), committed to bar_s.  Thread 0 only.
+    auto issue_scores = [&](uint32_t st) {
+        constexpr uint32_t IDESC = umma_idesc_bf16(128, MQ, false, false);
+        constexpr uint32_t HI = umma_desc_hi(1024u, 2u);
+        const uint32_t klo = umma_desc_lo(sbase + C::OFF_K + st * C::KV_TILE, 16u);
+        const uint32_t vlo = umma_desc_lo(sbase + C::OFF_V + st * C::KV_TILE, 16u);
+        const uint32_t qlo = umma_desc_lo(sbase + C::OFF_Q, 16u);
+        const uint32_t olo = umma_desc_lo(sbase + C::OFF_DO, 16u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t aoff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
+            const uint32_t boff = (uint32_t)(kk / 4) * (MQ * 128) + (uint32_t)(kk % 4) * 32u;
+            ptx::mma_bf16_ss(tmem + C::COL_S, umma_desc_join(klo + (aoff >> 4), HI),
+                             umma_desc_join(qlo + (boff >> 4), HI), IDESC, kk > 0 ? 1u : 0u);
+            ptx::mma_bf16_ss(tmem + C::COL_DP, umma_desc_join(vlo + (aoff >> 4), HI),
+                             umma_desc_join(olo + (boff >> 4), HI), IDESC, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar_s);
+    };
+    // dV = P^T dO and dK = dS^T Q (A in TMEM; B = the Q / dO tiles read MN-major) and
+    // dQ^T (+)= K^T dS^T (A = the K stage read MN-major; B = dS^T), committed to bar_g.
+    auto issue_grads = [&](uint32_t st, bool first_chunk) {
+        constexpr uint32_t IDESC_KV = umma_idesc_bf16(128, D, false, true);
+        constexpr uint32_t IDESC_Q = umma_idesc_bf16(D, MQ, true, true);
+        constexpr uint32_t HI_T = umma_desc_hi(1024u, 2u);
+        constexpr uint32_t P_LAYOUT = (C::P_ROW == 128) ? 2u : (C::P_ROW == 64) ? 4u : 6u;
+        constexpr uint32_t HI_DS = umma_desc_hi(8u * C::P_ROW, P_LAYOUT);
+        const uint32_t olo = umma_desc_lo(sbase + C::OFF_DO, (uint32_t)(MQ * 128));
+        const uint32_t qlo = umma_desc_lo(sbase + C::OFF_Q, (uint32_t)(MQ * 128));
+        const uint32_t klo = umma_desc_lo(sbase + C::OFF_K + st * C::KV_TILE, 128u * 128u);
+        const uint32_t dlo = umma_desc_lo(sbase + C::OFF_DS, (uint32_t)C::P_PANEL);
+#pragma unroll
+        for (int kk = 0; kk < MQ / 16; ++kk) {  // over the block's queries
+            ptx::mma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_P + (uint32_t)kk * 8u,
+                             umma_desc_join(olo + (uint32_t)(kk * 2048 >> 4), HI_T), IDESC_KV, kk > 0 ? 1u : 0u);
+            ptx::mma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DS + (uint32_t)kk * 8u,
+                             umma_desc_join(qlo + (uint32_t)(kk * 2048 >> 4), HI_T), IDESC_KV, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // over the chunk's keys
+            ptx::mma_bf16_ss(tmem + C::COL_DQ, umma_desc_join(klo + (uint32_t)(kk * 2048 >> 4), HI_T),
+                             umma_desc_join(dlo + (uint32_t)(kk * 16 * C::P_ROW >> 4), HI_DS), IDESC_Q,
+                             (!first_chunk || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(bar_g);
+    };
+
     uint32_t ph_s = 0, ph_g = 0;  // phases of the two MMA barriers
     bool failed = false;
     int64_t gcount = 0;  // chunks this block has processed (stage parity)
+    const uint32_t stg_row = (uint32_t)(t >> 4) * 2048u;  // this thread's 16-row box in a staged slice
+    const int srow = t & 15;                              // and its row in the box
     for (int64_t item = blockIdx.x; item < p.items && !failed; item += gridDim.x) {
         const int64_t bh = item / p.QB, qb = item - bh * p.QB;
         int64_t cnt = L;
@@ -172,18 +253,40 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
         const __nv_bfloat16* kb = p.k + bh * L * D;
         const __nv_bfloat16* vb = p.v + bh * L * D;
         const int64_t row0 = qb * MQ;
-        // key at list position j (checked), or 0 past the list
+        // key at list position j; -1 past the list or for an entry outside [0, L)
+        // (reported; such a row is loaded as zeros and gets no gradient)
         auto key_at = [&](int64_t j) -> int64_t {
-            if (j >= cnt) return 0;
+            if (j >= cnt) return -1;
             if (lst == nullptr) return j;
-            int32_t x = __ldg(lst + j);
+            const int32_t x = __ldg(lst + j);
             if (x < 0 || (int64_t)x >= L) {
                 atomicOr(&g_device_error, kErrBadIndex);
-                x = 0;
+                return -1;
             }
             return x;
         };
-        // ---- the block's Q and dO rows (zero past L), lse in log2 units and Delta
+        // K and V rows of chunk c into stage (gcount + c) & 1, one cp.async group.
+        // mykey = this thread's list entry of chunk c (-1: none); the warp loads the
+        // rows of its own 32 entries, PPR lanes per row, reading the keys by shuffle.
+        auto issue_chunk = [&](int64_t c, int32_t mykey) {
+            const uint32_t st = (uint32_t)((gcount + c) & 1);
+            const uint32_t kdst = sbase + C::OFF_K + st * C::KV_TILE, vdst = sbase + C::OFF_V + st * C::KV_TILE;
+            const int pc = lane % PPR;
+            const uint32_t panel = (uint32_t)(pc / 8) * (128u * 128u);
+#pragma unroll
+            for (int i = 0; i < 32 / RPI; ++i) {
+                const int rl = i * RPI + lane / PPR;  // row within the warp's 32
+                const int32_t key = __shfl_sync(0xffffffffu, mykey, rl);
+                const uint32_t off = panel + swz((uint32_t)(warp * 32 + rl), (uint32_t)(pc % 8), 128u);
+                const int64_t e = (int64_t)(key >= 0 ? key : 0) * D + pc * 8;
+                const uint32_t n = key >= 0 ? 16u : 0u;
+                ptx::cp_async_16(kdst + off, kb + e, n);
+                ptx::cp_async_16(vdst + off, vb + e, n);
+            }
+            ptx::cp_async_commit();
+        };
+        // ---- the block's Q and dO rows (zero past L), lse in log2 units and Delta;
+        //      then K/V of chunks 0 and 1
         {
             auto qrow = [&](int r) -> int64_t { return row0 + r < L ? row0 + r : -1; };
             load_rows(sbase + C::OFF_Q, MQ, p.q + bh * L * D, warp * (MQ / 4), MQ / 4, qrow);
@@ -195,47 +298,25 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
                 s_delta[t] = in ? p.delta[bh * L + row0 + t] : 0.f;
             }
         }
-        // K and V rows of chunk c into stage (gcount + c) & 1
-        auto issue_chunk = [&](int64_t c) {
-            const uint32_t st = (uint32_t)((gcount + c) & 1);
-            auto key_of = [&](int r) -> int64_t { return key_at(c * 128 + r); };
-            load_rows(sbase + C::OFF_K + st * C::KV_TILE, 128, kb, warp * 32, 32, key_of);
-            load_rows(sbase + C::OFF_V + st * C::KV_TILE, 128, vb, warp * 32, 32, key_of);
-            ptx::cp_async_commit();
-        };
-        issue_chunk(0);
+        // this thread's list entries of chunks c (key0) and c+1 (key1)
+        int32_t key0 = (int32_t)key_at(t);
+        int32_t key1 = nch > 1 ? (int32_t)key_at(128 + t) : -1;
+        issue_chunk(0, key0);
+        if (nch > 1) {
+            issue_chunk(1, key1);
+            ptx::cp_async_wait_group<1>();  // Q, dO and chunk 0 have landed
+        } else {
+            ptx::cp_async_wait_group<0>();
+        }
+        ptx::fence_proxy_async_smem();  // this thread's copies -> visible to the tensor core
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
+        if (t == 0) issue_scores((uint32_t)(gcount & 1));
         for (int64_t c = 0; c < nch; ++c) {
             const uint32_t st = (uint32_t)((gcount + c) & 1);
-            if (c + 1 < nch) {
-                issue_chunk(c + 1);
-                ptx::cp_async_wait_group<1>();  // all but the newest group have landed
-            } else {
-                ptx::cp_async_wait_group<0>();
-            }
-            ptx::fence_proxy_async_smem();  // this thread's copies -> visible to the tensor core
-            ptx::tc_fence_before();
-            __syncthreads();
-            ptx::tc_fence_after();
-            const uint32_t kst = sbase + C::OFF_K + st * C::KV_TILE;
-            const uint32_t vst = sbase + C::OFF_V + st * C::KV_TILE;
-            // ---- S^T = K Q^T and dP^T = V dO^T (K-major operands, M = 128 keys, N = MQ)
-            if (t == 0) {
-                constexpr uint32_t IDESC = umma_idesc_bf16(128, MQ, false, false);
-                constexpr uint32_t HI = umma_desc_hi(1024u, 2u);
-                const uint32_t klo = umma_desc_lo(kst, 16u), vlo = umma_desc_lo(vst, 16u);
-                const uint32_t qlo = umma_desc_lo(sbase + C::OFF_Q, 16u);
-                const uint32_t olo = umma_desc_lo(sbase + C::OFF_DO, 16u);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t aoff = (uint32_t)(kk / 4) * (128 * 128) + (uint32_t)(kk % 4) * 32u;
-                    const uint32_t boff = (uint32_t)(kk / 4) * (MQ * 128) + (uint32_t)(kk % 4) * 32u;
-                    ptx::mma_bf16_ss(tmem + C::COL_S, umma_desc_join(klo + (aoff >> 4), HI),
-                                     umma_desc_join(qlo + (boff >> 4), HI), IDESC, kk > 0 ? 1u : 0u);
-                    ptx::mma_bf16_ss(tmem + C::COL_DP, umma_desc_join(vlo + (aoff >> 4), HI),
-                                     umma_desc_join(olo + (boff >> 4), HI), IDESC, kk > 0 ? 1u : 0u);
-                }
-                ptx::mma_commit(bar_s);
-            }
+            // entry of chunk c+2, fetched now so that its latency hides behind the softmax
+            const int32_t key2 = c + 2 < nch ? (int32_t)key_at((c + 2) * 128 + t) : -1;
             if (!bounded_wait(bar_s, ph_s, abort_flag)) failed = true;
             ph_s ^= 1u;
             ptx::tc_fence_after();
@@ -289,68 +370,69 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
                 }
             }
             ptx::tmem_wait_st();
+            if (c + 1 < nch) ptx::cp_async_wait_group<0>();  // chunk c+1 (the newest group) has landed
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             __syncthreads();
             ptx::tc_fence_after();
-            // ---- dV = P^T dO and dK = dS^T Q (A in TMEM; B = the Q / dO tiles read
-            //      MN-major), dQ^T += K^T dS^T (A = the K stage read MN-major; B = dS^T)
+            // ---- gradient products of c, then the score products of c+1 behind them
             if (t == 0) {
-                constexpr uint32_t IDESC_KV = umma_idesc_bf16(128, D, false, true);
-                constexpr uint32_t IDESC_Q = umma_idesc_bf16(D, MQ, true, true);
-                constexpr uint32_t HI_T = umma_desc_hi(1024u, 2u);
-                constexpr uint32_t P_LAYOUT = (C::P_ROW == 128) ? 2u : (C::P_ROW == 64) ? 4u : 6u;
-                constexpr uint32_t HI_DS = umma_desc_hi(8u * C::P_ROW, P_LAYOUT);
-                const uint32_t olo = umma_desc_lo(sbase + C::OFF_DO, (uint32_t)(MQ * 128));
-                const uint32_t qlo = umma_desc_lo(sbase + C::OFF_Q, (uint32_t)(MQ * 128));
-                const uint32_t klo = umma_desc_lo(kst, 128u * 128u);
-                const uint32_t dlo = umma_desc_lo(sbase + C::OFF_DS, (uint32_t)C::P_PANEL);
-#pragma unroll
-                for (int kk = 0; kk < MQ / 16; ++kk) {  // over the block's queries
-                    ptx::mma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_P + (uint32_t)kk * 8u,
-                                     umma_desc_join(olo + (uint32_t)(kk * 2048 >> 4), HI_T), IDESC_KV,
-                                     kk > 0 ? 1u : 0u);
-                    ptx::mma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DS + (uint32_t)kk * 8u,
-                                     umma_desc_join(qlo + (uint32_t)(kk * 2048 >> 4), HI_T), IDESC_KV,
-                                     kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // over the chunk's keys
-                    ptx::mma_bf16_ss(tmem + C::COL_DQ, umma_desc_join(klo + (uint32_t)(kk * 2048 >> 4), HI_T),
-                                     umma_desc_join(dlo + (uint32_t)(kk * 16 * C::P_ROW >> 4), HI_DS), IDESC_Q,
-                                     (c > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(bar_g);
+                issue_grads(st, c == 0);
+                if (c + 1 < nch) issue_scores(st ^ 1u);
             }
             if (!bounded_wait(bar_g, ph_g, abort_flag)) failed = true;
             ph_g ^= 1u;
             ptx::tc_fence_after();
-            // ---- this key's dV and dK rows into the fp32 outputs (every lane reads TMEM;
-            //      only lanes of list keys store)
+            // stage st is free (both products of c are done): chunk c+2 goes there
+            if (c + 2 < nch) issue_chunk(c + 2, key2);
+            // ---- this chunk's dV and dK rows added to the outputs by the TMA unit
             {
-                const int64_t key = valid ? key_at(c * 128 + t) : -1;
-                float* dvr = p.dv + (bh * L + (key >= 0 ? key : 0)) * D;
-                float* dkr = p.dk + (bh * L + (key >= 0 ? key : 0)) * D;
+                const int64_t key = key0;
+                // a run: the 16 keys of this half-warp are consecutive and inside the head
+                const int64_t first = __shfl_sync(0xffffffffu, key, lane & 16);
+                const bool in_run = key >= 0 && key == first + (lane & 15) && first + 15 < L;
+                const uint32_t runs = __ballot_sync(0xffffffffu, in_run);
+                const bool seg_run = ((runs >> (lane & 16)) & 0xFFFFu) == 0xFFFFu;
 #pragma unroll 1
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     float a[32], b[32];
                     ptx::tmem_ld32(tmem + C::COL_DV + (uint32_t)c0 + lane_base, a);
                     ptx::tmem_ld32(tmem + C::COL_DK + (uint32_t)c0 + lane_base, b);
                     ptx::tmem_wait_ld();
-                    if (key >= 0) {
+                    ptx::bulk_wait_read_all();  // the staged slice before this one has been read
+                    __syncwarp();
+                    const uint32_t box_v = sbase + C::OFF_STG + stg_row, box_k = box_v + C::STG;
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4) {
-                            atomicAdd(reinterpret_cast<float4*>(dvr + c0 + e),
-                                      make_float4(a[e], a[e + 1], a[e + 2], a[e + 3]));
-                            atomicAdd(reinterpret_cast<float4*>(dkr + c0 + e),
-                                      make_float4(p.scale * b[e], p.scale * b[e + 1], p.scale * b[e + 2],
-                                                  p.scale * b[e + 3]));
+                    for (int j = 0; j < 8; ++j) {
+                        // runs: the box's 128B-swizzled layout; single rows: plain 128-byte rows
+                        const uint32_t off = seg_run ? swz((uint32_t)srow, (uint32_t)j, 128u)
+                                                     : (uint32_t)(srow * 128 + j * 16);
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box_v + off), "f"(a[4 * j]),
+                                     "f"(a[4 * j + 1]), "f"(a[4 * j + 2]), "f"(a[4 * j + 3])
+                                     : "memory");
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box_k + off),
+                                     "f"(p.scale * b[4 * j]), "f"(p.scale * b[4 * j + 1]), "f"(p.scale * b[4 * j + 2]),
+                                     "f"(p.scale * b[4 * j + 3])
+                                     : "memory");
+                    }
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (seg_run) {
+                        if ((lane & 15) == 0) {
+                            ptx::tma_reduce_add_3d(&p.tmap_dv, box_v, c0, (int32_t)first, (int32_t)bh);
+                            ptx::tma_reduce_add_3d(&p.tmap_dk, box_k, c0, (int32_t)first, (int32_t)bh);
+                            ptx::bulk_commit();
                         }
+                    } else if (key >= 0) {
+                        const int64_t off = (bh * L + key) * D + c0;
+                        ptx::bulk_reduce_add_f32(p.dv + off, box_v + (uint32_t)srow * 128u, 128u);
+                        ptx::bulk_reduce_add_f32(p.dk + off, box_k + (uint32_t)srow * 128u, 128u);
+                        ptx::bulk_commit();
                     }
                 }
             }
-            ptx::tc_fence_before();
-            __syncthreads();  // TMEM dV / dK, dS^T and the K stage are free for the next chunk
-            ptx::tc_fence_after();
+            key0 = key1;
+            key1 = key2;
         }
         gcount += nch;
         // ---- dQ rows of the block: dQ^T has D lanes x MQ columns (at D = 64 the M = 64
@@ -370,16 +452,18 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
             }
         }
         ptx::tc_fence_before();
-        // dQ^T read before the next block's first product overwrites it; leave together
+        // TMEM (dQ^T, dV, dK) read before the next block's products overwrite it; leave together
         failed = __syncthreads_or(failed);
         ptx::tc_fence_after();
     }
-    // drain: every MMA issued has completed before TMEM is freed
+    // drain: every MMA issued has completed before TMEM is freed, every copy and
+    // reduction before the block exits
     if (t == 0) {
         ptx::mma_commit(bar_drain);
         bounded_wait(bar_drain, 0u, abort_flag, /*honour_abort=*/false);
     }
     ptx::cp_async_wait_all();
+    ptx::bulk_wait_all();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();

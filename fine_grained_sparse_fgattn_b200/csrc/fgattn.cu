@@ -431,6 +431,21 @@ fgattn_status fgattn_masked_forward(const void* q, const void* k, const void* v,
 
 namespace {
 
+// fp32 gradient rows [B*H][L][d] as a 3-D map {d, L, B*H} in 32-column x 16-row boxes
+// (128B swizzle): the target of the backward kernel's box reductions.  Boxes never
+// reach past L, so a box never adds into another head's rows.
+bool encode_grad_map(CUtensorMap* m, float* base, int64_t BH, int64_t L, int64_t d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)(L * d * 4)};
+    const cuuint32_t box[3] = {32u, 16u, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int MQ>
 fgattn_status launch_bwd(const fgattn::BwdParams& prm, cudaStream_t s) {
     using C = fgattn::BwdCfg<D, MQ>;
@@ -483,20 +498,11 @@ fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const
     if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
     if (M != 16 && M != 32 && M != 64) return FGATTN_ERR_UNSUPPORTED;
     if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;
-    cudaStream_t s = (cudaStream_t)stream;
-    const int64_t rows = B * H * L;
-    const size_t grad_bytes = (size_t)rows * (size_t)d * sizeof(float);
-    if (cudaMemsetAsync(dk, 0, grad_bytes, s) != cudaSuccess) return FGATTN_ERR_CUDA;
-    if (cudaMemsetAsync(dv, 0, grad_bytes, s) != cudaSuccess) return FGATTN_ERR_CUDA;
-    const auto* ob = static_cast<const __nv_bfloat16*>(out);
-    const auto* gb = static_cast<const __nv_bfloat16*>(dout);
-    const unsigned dblocks = (unsigned)((rows + 7) / 8);
-    if (d == 128)
-        fgattn::fgattn_bwd_delta_kernel<128><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
-    else
-        fgattn::fgattn_bwd_delta_kernel<64><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
-    if (cudaPeekAtLastError() != cudaSuccess) return FGATTN_ERR_CUDA;
+    // tensor maps first: nothing is enqueued unless every host-side step succeeded
     fgattn::BwdParams prm;
+    if (!encode_grad_map(&prm.tmap_dk, dk, B * H, L, d) || !encode_grad_map(&prm.tmap_dv, dv, B * H, L, d))
+        return FGATTN_ERR_CUDA;
+    const auto* gb = static_cast<const __nv_bfloat16*>(dout);
     prm.q = static_cast<const __nv_bfloat16*>(q);
     prm.k = static_cast<const __nv_bfloat16*>(k);
     prm.v = static_cast<const __nv_bfloat16*>(v);
@@ -514,6 +520,18 @@ fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const
     prm.items = B * H * prm.QB;
     prm.scale = scale;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t rows = B * H * L;
+    const size_t grad_bytes = (size_t)rows * (size_t)d * sizeof(float);
+    if (cudaMemsetAsync(dk, 0, grad_bytes, s) != cudaSuccess) return FGATTN_ERR_CUDA;
+    if (cudaMemsetAsync(dv, 0, grad_bytes, s) != cudaSuccess) return FGATTN_ERR_CUDA;
+    const auto* ob = static_cast<const __nv_bfloat16*>(out);
+    const unsigned dblocks = (unsigned)((rows + 7) / 8);
+    if (d == 128)
+        fgattn::fgattn_bwd_delta_kernel<128><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
+    else
+        fgattn::fgattn_bwd_delta_kernel<64><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
+    if (cudaPeekAtLastError() != cudaSuccess) return FGATTN_ERR_CUDA;
     return d == 128 ? launch_bwd_m<128>(prm, M, s) : launch_bwd_m<64>(prm, M, s);
 }
 
