@@ -104,3 +104,33 @@ def test_backward_bad_index_is_flagged():
     idx[0, 0, 1, 5] = L + 7
     F.backward(q, k, v, out, g, lse, idx, cnt, M, N)
     assert F.device_error() & F.DEVERR_BAD_INDEX
+
+
+def test_backward_full_wan_layer(oracle):
+    """The Wan-480p-like layer at full size (B1 H40 L32760 d128, M64 N16, 70 %), in the
+    launch configuration the benchmark times: every head against two properties that
+    hold at any size (sum over keys of dk = 0, since every row's dS sums to zero; sum
+    over keys of dv = sum over queries of dO, since every row's probabilities sum to
+    one), and head 0 element by element against the oracle."""
+    w = W.get("wan480p")
+    dev = torch.device("cuda", 0)
+    q, k, v = W.make_qkv(w, 0)
+    g = W.random_grad(w.B, w.H, w.L, w.d, seed=17)
+    mask = W.make_mask(w, 0)
+    qd, kd, vd, gd = (t.to(dev) for t in (q, k, v, g))
+    idx, cnt = F.compact_mask(torch.from_numpy(mask.view(np.int32)).to(dev), w.B, w.H, w.L, w.M, w.N)
+    out, lse = F.forward(qd, kd, vd, idx, cnt, w.M, w.N, w.scale)
+    dq, dk, dv = F.backward(qd, kd, vd, out, gd, lse, idx, cnt, w.M, w.N, w.scale)
+    assert F.device_error() == 0
+    # properties, every head: relative to the size of the summed terms
+    sdk = dk.double().sum(dim=2)
+    assert (sdk.abs().max() / dk.double().abs().sum(dim=2).max()).item() < 1e-3
+    sdv = dv.double().sum(dim=2)
+    sg = gd.double().sum(dim=2)
+    assert ((sdv - sg).abs().max() / gd.double().abs().sum(dim=2).max()).item() < 1e-3
+    # head 0 against the oracle
+    h0 = range(1)
+    q0, k0, v0 = W.make_qkv(w, 0, heads=h0)
+    ref = oracle.backward(q0, k0, v0, g[:, :1], W.make_mask(w, 0, heads=h0), w.M, w.N, w.scale)
+    got = tuple(t[:, :1].cpu().double().numpy() for t in (dq, dk, dv))
+    print(compare_grads(got, ref))
