@@ -22,12 +22,16 @@
 // The adds happen in L2, with no per-thread atomics.
 //
 // One block of 128 threads per SM (persistent, round-robin over query blocks);
-// thread 0 also issues the MMAs.  Per chunk c: softmax(c); then the dV/dK/dQ
-// products of c and, behind them, the score products of c+1, so that the
-// tensor core computes S(c+1) while the threads write out dK/dV of c.  The K and
-// V rows of chunk c+2 are loaded with 16-byte cp.async copies into the stage of
-// chunk c once its products are done (two stages).  Every wait is bounded; on a
-// timeout the block sets the device error bit and stops.
+// thread 0 also issues the MMAs.  Per chunk c: the first half of softmax(c);
+// the second half of chunk c-1's dK/dV drain (its TMEM columns are intact until
+// the gradient products of c); the second half of softmax(c); then the dV/dK/dQ
+// products of c and, behind them, the score products of c+1; then the first
+// half of chunk c's drain while the tensor core computes S(c+1).  The TMA pushes
+// (128 KB per chunk, bound by the SM's L2 write port) thus overlap the softmax
+// and the score products.  The K and V rows of chunk c+2 are loaded with 16-byte
+// cp.async copies into the stage of chunk c once its products are done (two
+// stages).  Every wait is bounded; on a timeout the block sets the device error
+// bit and stops.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -84,6 +88,8 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, ui
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // every bulk group of this thread has finished reading its shared-memory source
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// all but this thread's most recent bulk group have finished reading their sources
+__device__ __forceinline__ void bulk_wait_read_but1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // every bulk group of this thread has completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -116,12 +122,12 @@ struct BwdCfg {
     static constexpr int P_TILE = KC * MQ * 2;
     static constexpr int STG = KC * 128;          // one staged 32-column slice of dV or dK (fp32)
     static constexpr int OFF_K = 0;                       // K stages [2]
-    static constexpr int OFF_V = OFF_K + 2 * KV_TILE;     // V stages [2]
-    static constexpr int OFF_Q = OFF_V + 2 * KV_TILE;
+    static constexpr int OFF_V = OFF_K + 2 * KV_TILE;     // V stage (one: only the score products read it)
+    static constexpr int OFF_Q = OFF_V + KV_TILE;
     static constexpr int OFF_DO = OFF_Q + Q_TILE;
     static constexpr int OFF_DS = OFF_DO + Q_TILE;        // dS^T, MN-major panels
-    static constexpr int OFF_STG = OFF_DS + P_TILE;       // dV slice, dK slice: [8 runs][16 rows][128 B]
-    static constexpr int OFF_LSE = OFF_STG + 2 * STG;     // float [MQ]: lse * log2(e) (+inf past L)
+    static constexpr int OFF_STG = OFF_DS + P_TILE;       // 2 slots x {dV slice, dK slice}: [8 runs][16 rows][128 B]
+    static constexpr int OFF_LSE = OFF_STG + 4 * STG;     // float [MQ]: lse * log2(e) (+inf past L)
     static constexpr int OFF_DELTA = OFF_LSE + MQ * 4;    // float [MQ]
     static constexpr int OFF_BAR = (OFF_DELTA + MQ * 4 + 7) / 8 * 8;  // s_done, g_done, drain
     static constexpr int OFF_TMEM = OFF_BAR + 3 * 8;
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
         constexpr uint32_t IDESC = umma_idesc_bf16(128, MQ, false, false);
         constexpr uint32_t HI = umma_desc_hi(1024u, 2u);
         const uint32_t klo = umma_desc_lo(sbase + C::OFF_K + st * C::KV_TILE, 16u);
-        const uint32_t vlo = umma_desc_lo(sbase + C::OFF_V + st * C::KV_TILE, 16u);
+        const uint32_t vlo = umma_desc_lo(sbase + C::OFF_V, 16u);
         const uint32_t qlo = umma_desc_lo(sbase + C::OFF_Q, 16u);
         const uint32_t olo = umma_desc_lo(sbase + C::OFF_DO, 16u);
 #pragma unroll
@@ -237,6 +243,7 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
     int64_t gcount = 0;  // chunks this block has processed (stage parity)
     const uint32_t stg_row = (uint32_t)(t >> 4) * 2048u;  // this thread's 16-row box in a staged slice
     const int srow = t & 15;                              // and its row in the box
+    uint32_t nsl = 0;                                     // slices this thread has staged
     for (int64_t item = blockIdx.x; item < p.items && !failed; item += gridDim.x) {
         const int64_t bh = item / p.QB, qb = item - bh * p.QB;
         int64_t cnt = L;
@@ -265,12 +272,11 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
             }
             return x;
         };
-        // K and V rows of chunk c into stage (gcount + c) & 1, one cp.async group.
-        // mykey = this thread's list entry of chunk c (-1: none); the warp loads the
-        // rows of its own 32 entries, PPR lanes per row, reading the keys by shuffle.
-        auto issue_chunk = [&](int64_t c, int32_t mykey) {
-            const uint32_t st = (uint32_t)((gcount + c) & 1);
-            const uint32_t kdst = sbase + C::OFF_K + st * C::KV_TILE, vdst = sbase + C::OFF_V + st * C::KV_TILE;
+        // K rows of chunk c into stage (gcount + c) & 1, or V rows into the V stage (one
+        // cp.async group).  mykey = this thread's list entry of chunk c (-1: none); the
+        // warp loads the rows of its own 32 entries, PPR lanes per row, reading the keys
+        // by shuffle.
+        auto issue_rows = [&](uint32_t dst, const __nv_bfloat16* src_base, int32_t mykey) {
             const int pc = lane % PPR;
             const uint32_t panel = (uint32_t)(pc / 8) * (128u * 128u);
 #pragma unroll
@@ -278,13 +284,14 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
                 const int rl = i * RPI + lane / PPR;  // row within the warp's 32
                 const int32_t key = __shfl_sync(0xffffffffu, mykey, rl);
                 const uint32_t off = panel + swz((uint32_t)(warp * 32 + rl), (uint32_t)(pc % 8), 128u);
-                const int64_t e = (int64_t)(key >= 0 ? key : 0) * D + pc * 8;
-                const uint32_t n = key >= 0 ? 16u : 0u;
-                ptx::cp_async_16(kdst + off, kb + e, n);
-                ptx::cp_async_16(vdst + off, vb + e, n);
+                ptx::cp_async_16(dst + off, src_base + (int64_t)(key >= 0 ? key : 0) * D + pc * 8, key >= 0 ? 16u : 0u);
             }
             ptx::cp_async_commit();
         };
+        auto issue_k = [&](int64_t c, int32_t mykey) {
+            issue_rows(sbase + C::OFF_K + (uint32_t)((gcount + c) & 1) * C::KV_TILE, kb, mykey);
+        };
+        auto issue_v = [&](int32_t mykey) { issue_rows(sbase + C::OFF_V, vb, mykey); };
         // ---- the block's Q and dO rows (zero past L), lse in log2 units and Delta;
         //      then K/V of chunks 0 and 1
         {
@@ -301,10 +308,11 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
         // this thread's list entries of chunks c (key0) and c+1 (key1)
         int32_t key0 = (int32_t)key_at(t);
         int32_t key1 = nch > 1 ? (int32_t)key_at(128 + t) : -1;
-        issue_chunk(0, key0);
+        issue_k(0, key0);
+        issue_v(key0);
         if (nch > 1) {
-            issue_chunk(1, key1);
-            ptx::cp_async_wait_group<1>();  // Q, dO and chunk 0 have landed
+            issue_k(1, key1);
+            ptx::cp_async_wait_group<1>();  // Q, dO and K, V of chunk 0 have landed
         } else {
             ptx::cp_async_wait_group<0>();
         }
@@ -313,18 +321,14 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
         __syncthreads();
         ptx::tc_fence_after();
         if (t == 0) issue_scores((uint32_t)(gcount & 1));
-        for (int64_t c = 0; c < nch; ++c) {
-            const uint32_t st = (uint32_t)((gcount + c) & 1);
-            // entry of chunk c+2, fetched now so that its latency hides behind the softmax
-            const int32_t key2 = c + 2 < nch ? (int32_t)key_at((c + 2) * 128 + t) : -1;
-            if (!bounded_wait(bar_s, ph_s, abort_flag)) failed = true;
-            ph_s ^= 1u;
-            ptx::tc_fence_after();
-            // ---- P^T and dS^T of this thread's key, up to 32 query columns at a time
+        // P^T and dS^T of this thread's key in chunk c for query columns [qa, qe), up to
+        // 32 at a time: TMEM (A operands, two queries per column) and, for dS^T, shared
+        // memory (B operand of dQ^T: MN-major, queries contiguous).
+        auto softmax_cols = [&](int64_t c, int qa, int qe) {
             const bool valid = c * 128 + t < cnt;
             constexpr int QW = MQ < 32 ? MQ : 32;
 #pragma unroll 1
-            for (int q0 = 0; q0 < MQ; q0 += QW) {
+            for (int q0 = qa; q0 < qe; q0 += QW) {
                 float sv[QW], dp[QW];
                 if constexpr (QW == 32) {
                     ptx::tmem_ld32(tmem + C::COL_S + (uint32_t)q0 + lane_base, sv);
@@ -349,7 +353,6 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
                     pp[j / 2] = *reinterpret_cast<uint32_t*>(&hp);
                     dd[j / 2] = *reinterpret_cast<uint32_t*>(&hd);
                 }
-                // P^T and dS^T rows of this key into TMEM (A operands: two queries per column)
                 if constexpr (QW == 32) {
                     ptx::tmem_st16u(tmem + C::COL_P + (uint32_t)(q0 / 2) + lane_base, pp);
                     ptx::tmem_st16u(tmem + C::COL_DS + (uint32_t)(q0 / 2) + lane_base, dd);
@@ -357,7 +360,6 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
                     ptx::tmem_st8u(tmem + C::COL_P + (uint32_t)(q0 / 2) + lane_base, pp);
                     ptx::tmem_st8u(tmem + C::COL_DS + (uint32_t)(q0 / 2) + lane_base, dd);
                 }
-                // the dS^T row into shared memory (B operand of dQ^T: MN-major, queries contiguous)
 #pragma unroll
                 for (int j = 0; j < QW; j += 8) {
                     const int chunk = (q0 + j) / 8;  // 16-byte chunk = 8 queries
@@ -369,8 +371,72 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
                                  : "memory");
                 }
             }
+        };
+        // 32-column slices [sa, se) of the chunk's dV and dK rows (this thread's key;
+        // -1: none) added to the outputs by the TMA unit, one slice at a time through
+        // the staging buffer.  run: the 16 keys of this half-warp are consecutive
+        // (first = the half's first key): one box per half-warp, else one row each.
+        auto drain = [&](int sa, int se, int32_t key, int32_t first, bool run) {
+#pragma unroll 1
+            for (int sl = sa; sl < se; ++sl) {
+                const int c0 = sl * 32;
+                float a[32], b[32];
+                ptx::tmem_ld32(tmem + C::COL_DV + (uint32_t)c0 + lane_base, a);
+                ptx::tmem_ld32(tmem + C::COL_DK + (uint32_t)c0 + lane_base, b);
+                ptx::tmem_wait_ld();
+                // slot (nsl & 1) was last filled two slices ago: every lane committed one
+                // bulk group per slice since, so "all but the newest group read" frees it
+                ptx::bulk_wait_read_but1();
+                __syncwarp();
+                const uint32_t box_v = sbase + C::OFF_STG + (nsl & 1u) * (2u * C::STG) + stg_row, box_k = box_v + C::STG;
+                ++nsl;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    // runs: the box's 128B-swizzled layout; single rows: plain 128-byte rows
+                    const uint32_t off = run ? swz((uint32_t)srow, (uint32_t)j, 128u) : (uint32_t)(srow * 128 + j * 16);
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box_v + off), "f"(a[4 * j]),
+                                 "f"(a[4 * j + 1]), "f"(a[4 * j + 2]), "f"(a[4 * j + 3])
+                                 : "memory");
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box_k + off), "f"(p.scale * b[4 * j]),
+                                 "f"(p.scale * b[4 * j + 1]), "f"(p.scale * b[4 * j + 2]), "f"(p.scale * b[4 * j + 3])
+                                 : "memory");
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (run) {
+                    if ((lane & 15) == 0) {
+                        ptx::tma_reduce_add_3d(&p.tmap_dv, box_v, c0, first, (int32_t)bh);
+                        ptx::tma_reduce_add_3d(&p.tmap_dk, box_k, c0, first, (int32_t)bh);
+                    }
+                } else if (key >= 0) {
+                    const int64_t off = (bh * L + key) * D + c0;
+                    ptx::bulk_reduce_add_f32(p.dv + off, box_v + (uint32_t)srow * 128u, 128u);
+                    ptx::bulk_reduce_add_f32(p.dk + off, box_k + (uint32_t)srow * 128u, 128u);
+                }
+                ptx::bulk_commit();  // one group per lane and slice, empty or not
+            }
+        };
+        // Per chunk c: softmax(c) in two halves with the second half of chunk c-1's
+        // dV/dK drain between them (its TMEM columns stay intact until the gradient
+        // products of c), then the products, then the first half of chunk c's drain.
+        constexpr int NS = D / 32;                         // 32-column slices of dV / dK
+        constexpr int QH = MQ >= 64 ? MQ / 2 : MQ;         // softmax columns before the drain
+        int32_t key_prev = -1, first_prev = 0;
+        bool run_prev = false;
+        for (int64_t c = 0; c < nch; ++c) {
+            const uint32_t st = (uint32_t)((gcount + c) & 1);
+            // entry of chunk c+2, fetched now so that its latency hides behind the softmax
+            const int32_t key2 = c + 2 < nch ? (int32_t)key_at((c + 2) * 128 + t) : -1;
+            if (!bounded_wait(bar_s, ph_s, abort_flag)) failed = true;
+            ph_s ^= 1u;
+            ptx::tc_fence_after();
+            // the score products of c are done with the V stage: V rows of chunk c+1
+            if (c + 1 < nch) issue_v(key1);
+            softmax_cols(c, 0, QH);
+            if (c > 0) drain(NS / 2, NS, key_prev, first_prev, run_prev);
+            if (QH < MQ) softmax_cols(c, QH, MQ);
             ptx::tmem_wait_st();
-            if (c + 1 < nch) ptx::cp_async_wait_group<0>();  // chunk c+1 (the newest group) has landed
+            if (c + 1 < nch) ptx::cp_async_wait_group<0>();  // K and V of chunk c+1 (the newest groups) have landed
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             __syncthreads();
@@ -383,57 +449,23 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
             if (!bounded_wait(bar_g, ph_g, abort_flag)) failed = true;
             ph_g ^= 1u;
             ptx::tc_fence_after();
-            // stage st is free (both products of c are done): chunk c+2 goes there
-            if (c + 2 < nch) issue_chunk(c + 2, key2);
-            // ---- this chunk's dV and dK rows added to the outputs by the TMA unit
+            // K stage st is free (both products of c are done): K rows of chunk c+2 go there
+            if (c + 2 < nch) issue_k(c + 2, key2);
+            // ---- first half of this chunk's dV / dK drain
             {
-                const int64_t key = key0;
-                // a run: the 16 keys of this half-warp are consecutive and inside the head
-                const int64_t first = __shfl_sync(0xffffffffu, key, lane & 16);
-                const bool in_run = key >= 0 && key == first + (lane & 15) && first + 15 < L;
+                const int32_t first = __shfl_sync(0xffffffffu, key0, lane & 16);
+                const bool in_run = key0 >= 0 && key0 == first + (lane & 15) && (int64_t)first + 15 < L;
                 const uint32_t runs = __ballot_sync(0xffffffffu, in_run);
-                const bool seg_run = ((runs >> (lane & 16)) & 0xFFFFu) == 0xFFFFu;
-#pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    float a[32], b[32];
-                    ptx::tmem_ld32(tmem + C::COL_DV + (uint32_t)c0 + lane_base, a);
-                    ptx::tmem_ld32(tmem + C::COL_DK + (uint32_t)c0 + lane_base, b);
-                    ptx::tmem_wait_ld();
-                    ptx::bulk_wait_read_all();  // the staged slice before this one has been read
-                    __syncwarp();
-                    const uint32_t box_v = sbase + C::OFF_STG + stg_row, box_k = box_v + C::STG;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        // runs: the box's 128B-swizzled layout; single rows: plain 128-byte rows
-                        const uint32_t off = seg_run ? swz((uint32_t)srow, (uint32_t)j, 128u)
-                                                     : (uint32_t)(srow * 128 + j * 16);
-                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box_v + off), "f"(a[4 * j]),
-                                     "f"(a[4 * j + 1]), "f"(a[4 * j + 2]), "f"(a[4 * j + 3])
-                                     : "memory");
-                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box_k + off),
-                                     "f"(p.scale * b[4 * j]), "f"(p.scale * b[4 * j + 1]), "f"(p.scale * b[4 * j + 2]),
-                                     "f"(p.scale * b[4 * j + 3])
-                                     : "memory");
-                    }
-                    ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                    if (seg_run) {
-                        if ((lane & 15) == 0) {
-                            ptx::tma_reduce_add_3d(&p.tmap_dv, box_v, c0, (int32_t)first, (int32_t)bh);
-                            ptx::tma_reduce_add_3d(&p.tmap_dk, box_k, c0, (int32_t)first, (int32_t)bh);
-                            ptx::bulk_commit();
-                        }
-                    } else if (key >= 0) {
-                        const int64_t off = (bh * L + key) * D + c0;
-                        ptx::bulk_reduce_add_f32(p.dv + off, box_v + (uint32_t)srow * 128u, 128u);
-                        ptx::bulk_reduce_add_f32(p.dk + off, box_k + (uint32_t)srow * 128u, 128u);
-                        ptx::bulk_commit();
-                    }
-                }
+                const bool run = ((runs >> (lane & 16)) & 0xFFFFu) == 0xFFFFu;
+                drain(0, NS / 2, key0, first, run);
+                key_prev = key0;
+                first_prev = first;
+                run_prev = run;
             }
             key0 = key1;
             key1 = key2;
         }
+        drain(NS / 2, NS, key_prev, first_prev, run_prev);  // second half of the last chunk
         gcount += nch;
         // ---- dQ rows of the block: dQ^T has D lanes x MQ columns (at D = 64 the M = 64
         //      accumulator holds row 16 * warp + lane in lanes 0..15 of each warp)
