@@ -355,8 +355,10 @@ def run_backward(args, w, F):
 
     peaks, peak_kind = load_peaks()
     achieved = flops_per_step / (bwd_ms * 1e-3) / 1e12
+    from fine_grained_sparse_fgattn_b200 import _build
+    traffic, _ = ncu_traffic(profile_key(w, args), _build.kernel_hash("bwd"), "fgattn_bwd")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                 "peak_kind": f"{peak_kind} bf16 burst", "kernel": f"fgattn_bwd_kernel<{d},{M}>",
                 "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "flops_per_launch": flops_per_step,
