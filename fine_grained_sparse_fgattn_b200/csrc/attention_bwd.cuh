@@ -21,17 +21,19 @@
 // 16 x 32 box reduction; any other row goes out as one 128-byte bulk reduction.
 // The adds happen in L2, with no per-thread atomics.
 //
-// One block of 128 threads per SM (persistent, round-robin over query blocks);
-// thread 0 also issues the MMAs.  Per chunk c: the first half of softmax(c);
-// the second half of chunk c-1's dK/dV drain (its TMEM columns are intact until
-// the gradient products of c); the second half of softmax(c); then the dV/dK/dQ
-// products of c and, behind them, the score products of c+1; then the first
-// half of chunk c's drain while the tensor core computes S(c+1).  The TMA pushes
-// (128 KB per chunk, bound by the SM's L2 write port) thus overlap the softmax
-// and the score products.  The K and V rows of chunk c+2 are loaded with 16-byte
-// cp.async copies into the stage of chunk c once its products are done (two
-// stages).  Every wait is bounded; on a timeout the block sets the device error
-// bit and stops.
+// One block of eight warps per SM (persistent, round-robin over query blocks).
+// A warp can only read the TMEM lane quarter (w % 4), so the two warps of a
+// quarter share its 32 keys and split the columns: the softmax's query halves,
+// dV (warps 0-3) and dK (warps 4-7), K rows and V rows; thread 0 also issues
+// the MMAs.  Per chunk c: softmax(c); the second half of chunk c-1's dK/dV drain
+// (its TMEM columns are intact until the gradient products of c); then the
+// dV/dK/dQ products of c and, behind them, the score products of c+1; then the
+// first half of chunk c's drain while the tensor core computes S(c+1).  The TMA
+// pushes (128 KB per chunk) thus overlap the softmax and the score products.  K
+// rows of chunk c+2 are loaded with 16-byte cp.async copies into the stage of
+// chunk c once its products are done (two K stages); V rows of chunk c+1 into
+// the single V stage once the score products of c are done.  Every wait is
+// bounded; on a timeout the block sets the device error bit and stops.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -44,7 +46,13 @@ namespace fgattn {
 
 namespace ptx {
 
-// 32 lanes x 8 / 16 consecutive 32-bit TMEM columns from raw words (packed bf16 pairs).
+// 32 lanes x 4 / 8 / 16 consecutive 32-bit TMEM columns from raw words (packed bf16 pairs).
+__device__ __forceinline__ void tmem_st4u(uint32_t taddr, const uint32_t (&r)[4]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&r)[8]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
                  "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
@@ -113,6 +121,7 @@ struct BwdCfg {
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(MQ == 16 || MQ == 32 || MQ == 64, "query block");
     static constexpr int KC = 128;                // keys per chunk
+    static constexpr int THREADS = 256;           // two warps per TMEM lane quarter
     static constexpr int ROW = D * 2;             // bytes per bf16 row
     static constexpr int KV_TILE = KC * ROW;      // one chunk of K or V rows
     static constexpr int Q_TILE = MQ * ROW;       // the block's Q or dO rows
@@ -146,7 +155,7 @@ struct BwdCfg {
 };
 
 template <int D, int MQ>
-__global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(BwdCfg<D, MQ>::THREADS, 1) fgattn_bwd_kernel(const __grid_constant__ BwdParams p) {
     using C = BwdCfg<D, MQ>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -155,8 +164,13 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
     const uint32_t bar_s = sbase + C::OFF_BAR, bar_g = bar_s + 8, bar_drain = bar_s + 16;
     float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
     float* s_delta = reinterpret_cast<float*>(smem + C::OFF_DELTA);
+    // Eight warps: warp w reads TMEM lanes 32 (w % 4) .. +31 (its quarter), so the two
+    // warps of a quarter share one chunk's 32 keys and split the columns: softmax
+    // query halves, dV (half 0) / dK (half 1), K rows (half 0) / V rows (half 1).
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int kt = quarter * 32 + lane;  // this thread's key row of a chunk = its TMEM lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int64_t L = p.L;
 
     if (warp == 0) {
@@ -191,8 +205,8 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
         }
     };
 
-    // S^T = K Q^T and dP^T = V dO^T of the chunk in stage st (K-major operands,
-    // M = 128 keys, N = MQ), committed to bar_s.  Thread 0 only.
+    // S^T = K Q^T and dP^T = V dO^T of the chunk whose K rows are in stage st (K-major
+    // operands, M = 128 keys, N = MQ), committed to bar_s.  Thread 0 only.
     auto issue_scores = [&](uint32_t st) {
         constexpr uint32_t IDESC = umma_idesc_bf16(128, MQ, false, false);
         constexpr uint32_t HI = umma_desc_hi(1024u, 2u);
@@ -240,10 +254,14 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
 
     uint32_t ph_s = 0, ph_g = 0;  // phases of the two MMA barriers
     bool failed = false;
-    int64_t gcount = 0;  // chunks this block has processed (stage parity)
-    const uint32_t stg_row = (uint32_t)(t >> 4) * 2048u;  // this thread's 16-row box in a staged slice
-    const int srow = t & 15;                              // and its row in the box
-    uint32_t nsl = 0;                                     // slices this thread has staged
+    int64_t gcount = 0;  // chunks this block has processed (K stage parity)
+    const uint32_t stg_row = (uint32_t)(kt >> 4) * 2048u + (half ? (uint32_t)C::STG : 0u);  // 16-row box, dV | dK
+    const int srow = kt & 15;  // this thread's row in the box
+    uint32_t nsl = 0;          // slices this thread has staged
+    const CUtensorMap* tmap_g = half ? &p.tmap_dk : &p.tmap_dv;
+    float* const grad = half ? p.dk : p.dv;
+    const float gscale = half ? p.scale : 1.f;
+    const uint32_t col_g = half ? C::COL_DK : C::COL_DV;
     for (int64_t item = blockIdx.x; item < p.items && !failed; item += gridDim.x) {
         const int64_t bh = item / p.QB, qb = item - bh * p.QB;
         int64_t cnt = L;
@@ -272,18 +290,18 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
             }
             return x;
         };
-        // K rows of chunk c into stage (gcount + c) & 1, or V rows into the V stage (one
-        // cp.async group).  mykey = this thread's list entry of chunk c (-1: none); the
-        // warp loads the rows of its own 32 entries, PPR lanes per row, reading the keys
-        // by shuffle.
+        // K rows (half 0) of chunk c into stage (gcount + c) & 1, or V rows (half 1)
+        // into the V stage, one cp.async group.  mykey = this thread's list entry of
+        // chunk c (-1: none); the warp loads the rows of its quarter's 32 entries, PPR
+        // lanes per row, reading the keys by shuffle.
         auto issue_rows = [&](uint32_t dst, const __nv_bfloat16* src_base, int32_t mykey) {
             const int pc = lane % PPR;
             const uint32_t panel = (uint32_t)(pc / 8) * (128u * 128u);
 #pragma unroll
             for (int i = 0; i < 32 / RPI; ++i) {
-                const int rl = i * RPI + lane / PPR;  // row within the warp's 32
+                const int rl = i * RPI + lane / PPR;  // row within the quarter's 32
                 const int32_t key = __shfl_sync(0xffffffffu, mykey, rl);
-                const uint32_t off = panel + swz((uint32_t)(warp * 32 + rl), (uint32_t)(pc % 8), 128u);
+                const uint32_t off = panel + swz((uint32_t)(quarter * 32 + rl), (uint32_t)(pc % 8), 128u);
                 ptx::cp_async_16(dst + off, src_base + (int64_t)(key >= 0 ? key : 0) * D + pc * 8, key >= 0 ? 16u : 0u);
             }
             ptx::cp_async_commit();
@@ -292,12 +310,12 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
             issue_rows(sbase + C::OFF_K + (uint32_t)((gcount + c) & 1) * C::KV_TILE, kb, mykey);
         };
         auto issue_v = [&](int32_t mykey) { issue_rows(sbase + C::OFF_V, vb, mykey); };
-        // ---- the block's Q and dO rows (zero past L), lse in log2 units and Delta;
-        //      then K/V of chunks 0 and 1
+        // ---- the block's Q (half 0) or dO (half 1) rows, zero past L; lse in log2 units
+        //      and Delta; K (half 0) / V (half 1) of chunk 0, and K of chunk 1
         {
             auto qrow = [&](int r) -> int64_t { return row0 + r < L ? row0 + r : -1; };
-            load_rows(sbase + C::OFF_Q, MQ, p.q + bh * L * D, warp * (MQ / 4), MQ / 4, qrow);
-            load_rows(sbase + C::OFF_DO, MQ, p.dout + bh * L * D, warp * (MQ / 4), MQ / 4, qrow);
+            load_rows(sbase + (half ? C::OFF_DO : C::OFF_Q), MQ, (half ? p.dout : p.q) + bh * L * D, quarter * (MQ / 4),
+                      MQ / 4, qrow);
             ptx::cp_async_commit();
             if (t < MQ) {
                 const bool in = row0 + t < L;
@@ -306,137 +324,135 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
             }
         }
         // this thread's list entries of chunks c (key0) and c+1 (key1)
-        int32_t key0 = (int32_t)key_at(t);
-        int32_t key1 = nch > 1 ? (int32_t)key_at(128 + t) : -1;
-        issue_k(0, key0);
-        issue_v(key0);
-        if (nch > 1) {
-            issue_k(1, key1);
-            ptx::cp_async_wait_group<1>();  // Q, dO and K, V of chunk 0 have landed
+        int32_t key0 = (int32_t)key_at(kt);
+        int32_t key1 = nch > 1 ? (int32_t)key_at(128 + kt) : -1;
+        if (half == 0) {
+            issue_k(0, key0);
+            if (nch > 1) {
+                issue_k(1, key1);
+                ptx::cp_async_wait_group<1>();  // Q and K of chunk 0 have landed
+            } else {
+                ptx::cp_async_wait_group<0>();
+            }
         } else {
-            ptx::cp_async_wait_group<0>();
+            issue_v(key0);
+            ptx::cp_async_wait_group<0>();  // dO and V of chunk 0 have landed
         }
         ptx::fence_proxy_async_smem();  // this thread's copies -> visible to the tensor core
         ptx::tc_fence_before();
         __syncthreads();
         ptx::tc_fence_after();
         if (t == 0) issue_scores((uint32_t)(gcount & 1));
-        // P^T and dS^T of this thread's key in chunk c for query columns [qa, qe), up to
-        // 32 at a time: TMEM (A operands, two queries per column) and, for dS^T, shared
-        // memory (B operand of dQ^T: MN-major, queries contiguous).
-        auto softmax_cols = [&](int64_t c, int qa, int qe) {
-            const bool valid = c * 128 + t < cnt;
-            constexpr int QW = MQ < 32 ? MQ : 32;
-#pragma unroll 1
-            for (int q0 = qa; q0 < qe; q0 += QW) {
-                float sv[QW], dp[QW];
-                if constexpr (QW == 32) {
-                    ptx::tmem_ld32(tmem + C::COL_S + (uint32_t)q0 + lane_base, sv);
-                    ptx::tmem_ld32(tmem + C::COL_DP + (uint32_t)q0 + lane_base, dp);
-                } else {
-                    ptx::tmem_ld16(tmem + C::COL_S + (uint32_t)q0 + lane_base, sv);
-                    ptx::tmem_ld16(tmem + C::COL_DP + (uint32_t)q0 + lane_base, dp);
-                }
-                ptx::tmem_wait_ld();
-                uint32_t pp[QW / 2], dd[QW / 2];
+        // P^T and dS^T of this thread's key in chunk c for this half's QW query columns:
+        // TMEM (A operands, two queries per column) and, for dS^T, shared memory (B
+        // operand of dQ^T: MN-major, queries contiguous).
+        constexpr int QW = MQ / 2;
+        auto softmax_half = [&](int64_t c) {
+            const bool valid = c * 128 + kt < cnt;
+            const int q0 = half * QW;
+            float sv[QW], dp[QW];
+            if constexpr (QW == 32) {
+                ptx::tmem_ld32(tmem + C::COL_S + (uint32_t)q0 + lane_base, sv);
+                ptx::tmem_ld32(tmem + C::COL_DP + (uint32_t)q0 + lane_base, dp);
+            } else if constexpr (QW == 16) {
+                ptx::tmem_ld16(tmem + C::COL_S + (uint32_t)q0 + lane_base, sv);
+                ptx::tmem_ld16(tmem + C::COL_DP + (uint32_t)q0 + lane_base, dp);
+            } else {
+                ptx::tmem_ld8(tmem + C::COL_S + (uint32_t)q0 + lane_base, sv);
+                ptx::tmem_ld8(tmem + C::COL_DP + (uint32_t)q0 + lane_base, dp);
+            }
+            ptx::tmem_wait_ld();
+            uint32_t pp[QW / 2], dd[QW / 2];
 #pragma unroll
-                for (int j = 0; j < QW; j += 2) {
-                    float pr[2], ds[2];
+            for (int j = 0; j < QW; j += 2) {
+                float pr[2], ds[2];
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int q = q0 + j + e;
-                        pr[e] = valid ? ptx::ex2(fmaf(sv[j + e], p.scale_log2, -s_lse[q])) : 0.f;
-                        ds[e] = pr[e] * (dp[j + e] - s_delta[q]);
-                    }
-                    __nv_bfloat162 hp = __floats2bfloat162_rn(pr[0], pr[1]);
-                    __nv_bfloat162 hd = __floats2bfloat162_rn(ds[0], ds[1]);
-                    pp[j / 2] = *reinterpret_cast<uint32_t*>(&hp);
-                    dd[j / 2] = *reinterpret_cast<uint32_t*>(&hd);
+                for (int e = 0; e < 2; ++e) {
+                    const int q = q0 + j + e;
+                    pr[e] = valid ? ptx::ex2(fmaf(sv[j + e], p.scale_log2, -s_lse[q])) : 0.f;
+                    ds[e] = pr[e] * (dp[j + e] - s_delta[q]);
                 }
-                if constexpr (QW == 32) {
-                    ptx::tmem_st16u(tmem + C::COL_P + (uint32_t)(q0 / 2) + lane_base, pp);
-                    ptx::tmem_st16u(tmem + C::COL_DS + (uint32_t)(q0 / 2) + lane_base, dd);
-                } else {
-                    ptx::tmem_st8u(tmem + C::COL_P + (uint32_t)(q0 / 2) + lane_base, pp);
-                    ptx::tmem_st8u(tmem + C::COL_DS + (uint32_t)(q0 / 2) + lane_base, dd);
-                }
+                __nv_bfloat162 hp = __floats2bfloat162_rn(pr[0], pr[1]);
+                __nv_bfloat162 hd = __floats2bfloat162_rn(ds[0], ds[1]);
+                pp[j / 2] = *reinterpret_cast<uint32_t*>(&hp);
+                dd[j / 2] = *reinterpret_cast<uint32_t*>(&hd);
+            }
+            if constexpr (QW == 32) {
+                ptx::tmem_st16u(tmem + C::COL_P + (uint32_t)(q0 / 2) + lane_base, pp);
+                ptx::tmem_st16u(tmem + C::COL_DS + (uint32_t)(q0 / 2) + lane_base, dd);
+            } else if constexpr (QW == 16) {
+                ptx::tmem_st8u(tmem + C::COL_P + (uint32_t)(q0 / 2) + lane_base, pp);
+                ptx::tmem_st8u(tmem + C::COL_DS + (uint32_t)(q0 / 2) + lane_base, dd);
+            } else {
+                ptx::tmem_st4u(tmem + C::COL_P + (uint32_t)(q0 / 2) + lane_base, pp);
+                ptx::tmem_st4u(tmem + C::COL_DS + (uint32_t)(q0 / 2) + lane_base, dd);
+            }
 #pragma unroll
-                for (int j = 0; j < QW; j += 8) {
-                    const int chunk = (q0 + j) / 8;  // 16-byte chunk = 8 queries
-                    const int panel = chunk / C::P_CPR;
-                    const uint32_t addr = sbase + C::OFF_DS + (uint32_t)panel * C::P_PANEL +
-                                          swz((uint32_t)t, (uint32_t)(chunk % C::P_CPR), (uint32_t)C::P_ROW);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dd[j / 2]),
-                                 "r"(dd[j / 2 + 1]), "r"(dd[j / 2 + 2]), "r"(dd[j / 2 + 3])
-                                 : "memory");
-                }
+            for (int j = 0; j < QW; j += 8) {
+                const int chunk = (q0 + j) / 8;  // 16-byte chunk = 8 queries
+                const int panel = chunk / C::P_CPR;
+                const uint32_t addr = sbase + C::OFF_DS + (uint32_t)panel * C::P_PANEL +
+                                      swz((uint32_t)kt, (uint32_t)(chunk % C::P_CPR), (uint32_t)C::P_ROW);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dd[j / 2]), "r"(dd[j / 2 + 1]),
+                             "r"(dd[j / 2 + 2]), "r"(dd[j / 2 + 3])
+                             : "memory");
             }
         };
-        // 32-column slices [sa, se) of the chunk's dV and dK rows (this thread's key;
-        // -1: none) added to the outputs by the TMA unit, one slice at a time through
-        // the staging buffer.  run: the 16 keys of this half-warp are consecutive
-        // (first = the half's first key): one box per half-warp, else one row each.
+        // 32-column slices [sa, se) of this half's gradient (dV or dK) rows of the
+        // chunk (this thread's key; -1: none) added to the output by the TMA unit,
+        // through two staging slots.  run: the 16 keys of this half-warp are
+        // consecutive (first = the half-warp's first key): one box per half-warp,
+        // else one 128-byte row each.
         auto drain = [&](int sa, int se, int32_t key, int32_t first, bool run) {
 #pragma unroll 1
             for (int sl = sa; sl < se; ++sl) {
                 const int c0 = sl * 32;
-                float a[32], b[32];
-                ptx::tmem_ld32(tmem + C::COL_DV + (uint32_t)c0 + lane_base, a);
-                ptx::tmem_ld32(tmem + C::COL_DK + (uint32_t)c0 + lane_base, b);
+                float a[32];
+                ptx::tmem_ld32(tmem + col_g + (uint32_t)c0 + lane_base, a);
                 ptx::tmem_wait_ld();
                 // slot (nsl & 1) was last filled two slices ago: every lane committed one
                 // bulk group per slice since, so "all but the newest group read" frees it
                 ptx::bulk_wait_read_but1();
                 __syncwarp();
-                const uint32_t box_v = sbase + C::OFF_STG + (nsl & 1u) * (2u * C::STG) + stg_row, box_k = box_v + C::STG;
+                const uint32_t box = sbase + C::OFF_STG + (nsl & 1u) * (2u * C::STG) + stg_row;
                 ++nsl;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     // runs: the box's 128B-swizzled layout; single rows: plain 128-byte rows
                     const uint32_t off = run ? swz((uint32_t)srow, (uint32_t)j, 128u) : (uint32_t)(srow * 128 + j * 16);
-                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box_v + off), "f"(a[4 * j]),
-                                 "f"(a[4 * j + 1]), "f"(a[4 * j + 2]), "f"(a[4 * j + 3])
-                                 : "memory");
-                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box_k + off), "f"(p.scale * b[4 * j]),
-                                 "f"(p.scale * b[4 * j + 1]), "f"(p.scale * b[4 * j + 2]), "f"(p.scale * b[4 * j + 3])
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box + off), "f"(gscale * a[4 * j]),
+                                 "f"(gscale * a[4 * j + 1]), "f"(gscale * a[4 * j + 2]), "f"(gscale * a[4 * j + 3])
                                  : "memory");
                 }
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
                 if (run) {
-                    if ((lane & 15) == 0) {
-                        ptx::tma_reduce_add_3d(&p.tmap_dv, box_v, c0, first, (int32_t)bh);
-                        ptx::tma_reduce_add_3d(&p.tmap_dk, box_k, c0, first, (int32_t)bh);
-                    }
+                    if ((lane & 15) == 0) ptx::tma_reduce_add_3d(tmap_g, box, c0, first, (int32_t)bh);
                 } else if (key >= 0) {
-                    const int64_t off = (bh * L + key) * D + c0;
-                    ptx::bulk_reduce_add_f32(p.dv + off, box_v + (uint32_t)srow * 128u, 128u);
-                    ptx::bulk_reduce_add_f32(p.dk + off, box_k + (uint32_t)srow * 128u, 128u);
+                    ptx::bulk_reduce_add_f32(grad + (bh * L + key) * D + c0, box + (uint32_t)srow * 128u, 128u);
                 }
                 ptx::bulk_commit();  // one group per lane and slice, empty or not
             }
         };
-        // Per chunk c: softmax(c) in two halves with the second half of chunk c-1's
-        // dV/dK drain between them (its TMEM columns stay intact until the gradient
-        // products of c), then the products, then the first half of chunk c's drain.
-        constexpr int NS = D / 32;                         // 32-column slices of dV / dK
-        constexpr int QH = MQ >= 64 ? MQ / 2 : MQ;         // softmax columns before the drain
+        // Per chunk c: softmax(c), then the second half of chunk c-1's drain (its TMEM
+        // columns stay intact until the gradient products of c), then the products,
+        // then the first half of chunk c's drain while the tensor core computes S(c+1).
+        constexpr int NS = D / 32;  // 32-column slices of dV / dK
         int32_t key_prev = -1, first_prev = 0;
         bool run_prev = false;
         for (int64_t c = 0; c < nch; ++c) {
             const uint32_t st = (uint32_t)((gcount + c) & 1);
             // entry of chunk c+2, fetched now so that its latency hides behind the softmax
-            const int32_t key2 = c + 2 < nch ? (int32_t)key_at((c + 2) * 128 + t) : -1;
+            const int32_t key2 = c + 2 < nch ? (int32_t)key_at((c + 2) * 128 + kt) : -1;
             if (!bounded_wait(bar_s, ph_s, abort_flag)) failed = true;
             ph_s ^= 1u;
             ptx::tc_fence_after();
             // the score products of c are done with the V stage: V rows of chunk c+1
-            if (c + 1 < nch) issue_v(key1);
-            softmax_cols(c, 0, QH);
+            if (half == 1 && c + 1 < nch) issue_v(key1);
+            softmax_half(c);
             if (c > 0) drain(NS / 2, NS, key_prev, first_prev, run_prev);
-            if (QH < MQ) softmax_cols(c, QH, MQ);
             ptx::tmem_wait_st();
-            if (c + 1 < nch) ptx::cp_async_wait_group<0>();  // K and V of chunk c+1 (the newest groups) have landed
+            if (c + 1 < nch) ptx::cp_async_wait_group<0>();  // K or V of chunk c+1 (the newest group) has landed
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             __syncthreads();
@@ -450,7 +466,7 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
             ph_g ^= 1u;
             ptx::tc_fence_after();
             // K stage st is free (both products of c are done): K rows of chunk c+2 go there
-            if (c + 2 < nch) issue_k(c + 2, key2);
+            if (half == 0 && c + 2 < nch) issue_k(c + 2, key2);
             // ---- first half of this chunk's dV / dK drain
             {
                 const int32_t first = __shfl_sync(0xffffffffu, key0, lane & 16);
@@ -468,10 +484,11 @@ __global__ void __launch_bounds__(128, 1) fgattn_bwd_kernel(const __grid_constan
         drain(NS / 2, NS, key_prev, first_prev, run_prev);  // second half of the last chunk
         gcount += nch;
         // ---- dQ rows of the block: dQ^T has D lanes x MQ columns (at D = 64 the M = 64
-        //      accumulator holds row 16 * warp + lane in lanes 0..15 of each warp)
-        const int dt = (D == 128) ? t : ((lane < 16) ? warp * 16 + lane : -1);
+        //      accumulator holds row 16 * quarter + lane in lanes 0..15 of each quarter);
+        //      each half reads its MQ / 2 columns
+        const int dt = (D == 128) ? kt : ((lane < 16) ? quarter * 16 + lane : -1);
 #pragma unroll 1
-        for (int q0 = 0; q0 < MQ; q0 += 8) {
+        for (int q0 = half * (MQ / 2); q0 < (half + 1) * (MQ / 2); q0 += 8) {
             float o[8];
             ptx::tmem_ld8(tmem + C::COL_DQ + (uint32_t)q0 + lane_base, o);
             ptx::tmem_wait_ld();

@@ -463,7 +463,7 @@ fgattn_status launch_bwd(const fgattn::BwdParams& prm, cudaStream_t s) {
     const int sms = current_sms();
     if (sms <= 0) return FGATTN_ERR_CUDA;
     const int64_t grid = prm.items < sms ? prm.items : sms;
-    kernel<<<(unsigned)grid, 128, smem, s>>>(prm);
+    kernel<<<(unsigned)grid, C::THREADS, smem, s>>>(prm);
     return cudaPeekAtLastError() == cudaSuccess ? FGATTN_OK : FGATTN_ERR_CUDA;
 }
 
