@@ -111,7 +111,10 @@ struct alignas(64) BwdParams {
     const int32_t* kept_idx;                 // [items][cap], or null: every key kept
     const int32_t* kept_cnt;                 // [items]
     float *dq, *dk, *dv;                     // fp32 [B][H][L][D]; dk and dv accumulate (zeroed first)
-    int64_t cap, L, QB, items;
+    int64_t cap, L;
+    int64_t QB;      // query blocks of the lists (M rows each) per (b, h)
+    int64_t msplit;  // M / MQ: a 128-row block runs as two 64-row halves over one list
+    int64_t items;   // B * H * QB * msplit
     float scale;       // softmax scale
     float scale_log2;  // scale * log2(e)
 };
@@ -263,21 +266,22 @@ __global__ void __launch_bounds__(BwdCfg<D, MQ>::THREADS, 1) fgattn_bwd_kernel(c
     const float gscale = half ? p.scale : 1.f;
     const uint32_t col_g = half ? C::COL_DK : C::COL_DV;
     for (int64_t item = blockIdx.x; item < p.items && !failed; item += gridDim.x) {
-        const int64_t bh = item / p.QB, qb = item - bh * p.QB;
+        const int64_t blk = item / p.msplit;  // (b, h, qb) of the list
+        const int64_t bh = blk / p.QB, qb = blk - bh * p.QB;
         int64_t cnt = L;
         const int32_t* lst = nullptr;
         if (p.kept_idx != nullptr) {
-            cnt = p.kept_cnt[item];
+            cnt = p.kept_cnt[blk];
             if (cnt < 1 || cnt > p.cap) {
                 if (t == 0) atomicOr(&g_device_error, kErrBadCount);
                 cnt = cnt < 1 ? 1 : p.cap;
             }
-            lst = p.kept_idx + item * p.cap;
+            lst = p.kept_idx + blk * p.cap;
         }
         const int64_t nch = (cnt + 127) / 128;
         const __nv_bfloat16* kb = p.k + bh * L * D;
         const __nv_bfloat16* vb = p.v + bh * L * D;
-        const int64_t row0 = qb * MQ;
+        const int64_t row0 = (qb * p.msplit + (item - blk * p.msplit)) * MQ;  // this item's first query row
         // key at list position j; -1 past the list or for an entry outside [0, L)
         // (reported; such a row is loaded as zeros and gets no gradient)
         auto key_at = [&](int64_t j) -> int64_t {

@@ -496,7 +496,7 @@ fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const
         return FGATTN_ERR_INVALID_ARG;
     if (kept_idx && (cap < L || (cap & 3))) return FGATTN_ERR_CAPACITY;
     if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
-    if (M != 16 && M != 32 && M != 64) return FGATTN_ERR_UNSUPPORTED;
+    if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
     if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;
     // tensor maps first: nothing is enqueued unless every host-side step succeeded
     fgattn::BwdParams prm;
@@ -516,8 +516,12 @@ fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const
     prm.dv = dv;
     prm.cap = kept_idx ? cap : L;
     prm.L = L;
+    // 128-row blocks run as two 64-row halves over the block's list (the kernel's
+    // TMEM holds at most 64 query columns next to the dK/dV accumulators)
+    const int64_t MQ = M > 64 ? 64 : M;
     prm.QB = (L + M - 1) / M;
-    prm.items = B * H * prm.QB;
+    prm.msplit = M / MQ;
+    prm.items = B * H * prm.QB * prm.msplit;
     prm.scale = scale;
     prm.scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t s = (cudaStream_t)stream;
@@ -532,7 +536,7 @@ fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const
     else
         fgattn::fgattn_bwd_delta_kernel<64><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
     if (cudaPeekAtLastError() != cudaSuccess) return FGATTN_ERR_CUDA;
-    return d == 128 ? launch_bwd_m<128>(prm, M, s) : launch_bwd_m<64>(prm, M, s);
+    return d == 128 ? launch_bwd_m<128>(prm, MQ, s) : launch_bwd_m<64>(prm, MQ, s);
 }
 
 fgattn_status fgattn_device_error(fgattn_stream_t stream, int clear, uint32_t* bits) {

@@ -175,12 +175,14 @@ fgattn_status fgattn_masked_forward(const void* q, const void* k, const void* v,
  *                            block keeps get zeros)
  *   delta               out  device fp32 [B][H][L]: workspace owned by the
  *                            caller; holds delta_i on return
- * Supported: d in {64, 128}, M in {16, 32, 64}, any N >= 1, any L >= 1.
+ * Supported: d in {64, 128}, M in {16, 32, 64, 128} (a 128-row block runs as
+ * two 64-row halves over its list), any N >= 1, any L >= 1.
  * P and ds are rounded to bf16 for the tensor-core products; accumulation in
  * fp32.  dk and dv are accumulated with float atomics (many query blocks keep
  * one key), so their last bits depend on the order the blocks run in; dq is
  * deterministic.  Errors: INVALID_ARG, UNSUPPORTED, CAPACITY, CUDA; device-side
- * problems as for fgattn_forward.
+ * problems as for fgattn_forward, except that a kept_idx entry outside [0, L)
+ * (flagged BAD_INDEX) is read as a zero row and receives no gradient.
  */
 fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
                               const float* lse, const int32_t* kept_idx, const int32_t* kept_cnt, int64_t cap,

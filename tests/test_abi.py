@@ -168,7 +168,7 @@ def test_header_declares_backward():
     (dict(cap=63), F.ERR_CAPACITY),
     (dict(d=96), F.ERR_UNSUPPORTED),
     (dict(d=80), F.ERR_UNSUPPORTED),
-    (dict(M=128), F.ERR_UNSUPPORTED),
+    (dict(M=256), F.ERR_UNSUPPORTED),
     (dict(M=48), F.ERR_UNSUPPORTED),
 ])
 def test_backward_rejects(kw, status):

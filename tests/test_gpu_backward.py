@@ -72,6 +72,9 @@ CASES = [
     (16, 64, 16, 1, 0.3, 1), (37, 128, 16, 3, 0.5, 2), (300, 64, 32, 4, 0.3, 2), (257, 128, 64, 1, 0.4, 1),
     (700, 128, 64, 16, 0.3, 1), (640, 128, 32, 64, 0.5, 1), (200, 64, 64, 2, 0.6, 1), (383, 128, 16, 1, 1.0, 1),
     (128, 128, 64, 128, 0.0, 1), (97, 64, 16, 100, 0.5, 1), (1000, 64, 64, 33, 0.1, 1), (513, 128, 32, 7, 0.25, 2),
+    # 128-row blocks (two 64-row halves over one list): ragged last block, a last block
+    # whose second half is past L, one block
+    (700, 128, 128, 16, 0.3, 1), (450, 64, 128, 5, 0.4, 2), (100, 128, 128, 64, 0.5, 1),
 ]
 
 
@@ -80,7 +83,7 @@ def test_backward_matches_oracle(oracle, L, d, M, N, density, H):
     print(backward_case(oracle, L, d, M, N, density, H, seed=L * 5 + d + M + N))
 
 
-@pytest.mark.parametrize("M,d", [(16, 64), (64, 128)])
+@pytest.mark.parametrize("M,d", [(16, 64), (64, 128), (128, 128)])
 def test_backward_dense_run(oracle, M, d):
     """No lists: every key kept, the same kernel reading keys 0 .. L-1."""
     print(backward_case(oracle, 301, d, M, 16, 1.0, 2, seed=11, dense=True))
