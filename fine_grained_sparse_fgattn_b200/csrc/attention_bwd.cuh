@@ -121,11 +121,15 @@ struct alignas(64) BwdParams {
 
 template <int D, int MQ>
 struct BwdCfg {
-    static_assert(D == 64 || D == 128, "head dim");
+    static_assert(D == 64 || D == 96 || D == 128, "head dim");
     static_assert(MQ == 16 || MQ == 32 || MQ == 64, "query block");
+    // At D = 96 the tiles are 128 columns wide with columns 96..127 zero: the dV/dK
+    // products run with N = 128 and the dQ^T product with M = 128 (the shapes
+    // tcgen05 offers), and the padded columns are never stored.
+    static constexpr int DP = D == 96 ? 128 : D;
     static constexpr int KC = 128;                // keys per chunk
     static constexpr int THREADS = 256;           // two warps per TMEM lane quarter
-    static constexpr int ROW = D * 2;             // bytes per bf16 row
+    static constexpr int ROW = DP * 2;            // bytes per bf16 row of a tile
     static constexpr int KV_TILE = KC * ROW;      // one chunk of K or V rows
     static constexpr int Q_TILE = MQ * ROW;       // the block's Q or dO rows
     static constexpr int P_ROW = (MQ * 2 < 128) ? MQ * 2 : 128;  // bytes per key row of a dS^T panel
@@ -149,9 +153,9 @@ struct BwdCfg {
     static_assert(SMEM_REQUEST <= 227 * 1024, "shared memory");
     static_assert(OFF_STG % 1024 == 0, "staged boxes need 1024-byte aligned 128B-swizzle atoms");
     // TMEM columns: S^T, dP^T (MQ fp32 each), P^T and dS^T (MQ / 2 packed bf16 pairs
-    // each), dV and dK (D each, M = 128), dQ^T (MQ columns, M = D)
+    // each), dV and dK (DP each, M = 128), dQ^T (MQ columns, M = DP)
     static constexpr uint32_t COL_S = 0, COL_DP = MQ, COL_P = 2 * MQ, COL_DS = COL_P + MQ / 2;
-    static constexpr uint32_t COL_DV = COL_DS + MQ / 2, COL_DK = COL_DV + D, COL_DQ = COL_DK + D;
+    static constexpr uint32_t COL_DV = COL_DS + MQ / 2, COL_DK = COL_DV + DP, COL_DQ = COL_DK + DP;
     static constexpr uint32_t COLS_USED = COL_DQ + MQ;
     static constexpr uint32_t TMEM_COLS = COLS_USED <= 128 ? 128 : COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "TMEM columns");
@@ -195,16 +199,17 @@ __global__ void __launch_bounds__(BwdCfg<D, MQ>::THREADS, 1) fgattn_bwd_kernel(c
     // Rows r0 .. r0+nrows of a K-major 128B-swizzled tile (64-column panels of prow
     // rows) from base[key_of(r)] (zero-filled where key_of returns -1): one 16-byte
     // piece per lane, PPR lanes per row.
-    constexpr int PPR = D / 8;
+    constexpr int PPR = C::DP / 8;
     constexpr int RPI = 32 / PPR;  // rows per warp instruction
     auto load_rows = [&](uint32_t dst, int prow, const __nv_bfloat16* base, int r0, int nrows, auto key_of) {
         for (int i = 0; i < nrows / RPI; ++i) {
             const int r = r0 + i * RPI + lane / PPR;
             const int pc = lane % PPR;
             const int64_t key = key_of(r);
-            const __nv_bfloat16* src = base + (key >= 0 ? key : 0) * D + pc * 8;
+            const bool in = key >= 0 && pc * 8 < D;  // padded columns read as zeros
+            const __nv_bfloat16* src = base + (in ? key * D + pc * 8 : 0);
             ptx::cp_async_16(dst + (uint32_t)(pc / 8) * (uint32_t)(prow * 128) + swz((uint32_t)r, (uint32_t)(pc % 8), 128u),
-                             src, key >= 0 ? 16u : 0u);
+                             src, in ? 16u : 0u);
         }
     };
 
@@ -231,8 +236,8 @@ __global__ void __launch_bounds__(BwdCfg<D, MQ>::THREADS, 1) fgattn_bwd_kernel(c
     // dV = P^T dO and dK = dS^T Q (A in TMEM; B = the Q / dO tiles read MN-major) and
     // dQ^T (+)= K^T dS^T (A = the K stage read MN-major; B = dS^T), committed to bar_g.
     auto issue_grads = [&](uint32_t st, bool first_chunk) {
-        constexpr uint32_t IDESC_KV = umma_idesc_bf16(128, D, false, true);
-        constexpr uint32_t IDESC_Q = umma_idesc_bf16(D, MQ, true, true);
+        constexpr uint32_t IDESC_KV = umma_idesc_bf16(128, C::DP, false, true);
+        constexpr uint32_t IDESC_Q = umma_idesc_bf16(C::DP, MQ, true, true);
         constexpr uint32_t HI_T = umma_desc_hi(1024u, 2u);
         constexpr uint32_t P_LAYOUT = (C::P_ROW == 128) ? 2u : (C::P_ROW == 64) ? 4u : 6u;
         constexpr uint32_t HI_DS = umma_desc_hi(8u * C::P_ROW, P_LAYOUT);
@@ -305,8 +310,9 @@ __global__ void __launch_bounds__(BwdCfg<D, MQ>::THREADS, 1) fgattn_bwd_kernel(c
             for (int i = 0; i < 32 / RPI; ++i) {
                 const int rl = i * RPI + lane / PPR;  // row within the quarter's 32
                 const int32_t key = __shfl_sync(0xffffffffu, mykey, rl);
+                const bool in = key >= 0 && pc * 8 < D;  // padded columns read as zeros
                 const uint32_t off = panel + swz((uint32_t)(quarter * 32 + rl), (uint32_t)(pc % 8), 128u);
-                ptx::cp_async_16(dst + off, src_base + (int64_t)(key >= 0 ? key : 0) * D + pc * 8, key >= 0 ? 16u : 0u);
+                ptx::cp_async_16(dst + off, src_base + (in ? (int64_t)key * D + pc * 8 : 0), in ? 16u : 0u);
             }
             ptx::cp_async_commit();
         };
@@ -488,9 +494,10 @@ __global__ void __launch_bounds__(BwdCfg<D, MQ>::THREADS, 1) fgattn_bwd_kernel(c
         drain(NS / 2, NS, key_prev, first_prev, run_prev);  // second half of the last chunk
         gcount += nch;
         // ---- dQ rows of the block: dQ^T has D lanes x MQ columns (at D = 64 the M = 64
-        //      accumulator holds row 16 * quarter + lane in lanes 0..15 of each quarter);
+        //      accumulator holds row 16 * quarter + lane in lanes 0..15 of each quarter;
+        //      at D = 96 lanes 96..127 hold the zero padding);
         //      each half reads its MQ / 2 columns
-        const int dt = (D == 128) ? kt : ((lane < 16) ? quarter * 16 + lane : -1);
+        const int dt = (C::DP == 128) ? (kt < D ? kt : -1) : ((lane < 16) ? quarter * 16 + lane : -1);
 #pragma unroll 1
         for (int q0 = half * (MQ / 2); q0 < (half + 1) * (MQ / 2); q0 += 8) {
             float o[8];

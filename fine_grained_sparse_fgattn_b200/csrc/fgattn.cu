@@ -495,7 +495,7 @@ fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const
         (kept_idx && (reinterpret_cast<uintptr_t>(kept_idx) & 3u)))
         return FGATTN_ERR_INVALID_ARG;
     if (kept_idx && (cap < L || (cap & 3))) return FGATTN_ERR_CAPACITY;
-    if (d != 64 && d != 128) return FGATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 96 && d != 128) return FGATTN_ERR_UNSUPPORTED;
     if (M != 16 && M != 32 && M != 64 && M != 128) return FGATTN_ERR_UNSUPPORTED;
     if (B * H * L > INT32_MAX) return FGATTN_ERR_UNSUPPORTED;
     // tensor maps first: nothing is enqueued unless every host-side step succeeded
@@ -533,9 +533,12 @@ fgattn_status fgattn_backward(const void* q, const void* k, const void* v, const
     const unsigned dblocks = (unsigned)((rows + 7) / 8);
     if (d == 128)
         fgattn::fgattn_bwd_delta_kernel<128><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
+    else if (d == 96)
+        fgattn::fgattn_bwd_delta_kernel<96><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
     else
         fgattn::fgattn_bwd_delta_kernel<64><<<dblocks, 256, 0, s>>>(ob, gb, delta, rows);
     if (cudaPeekAtLastError() != cudaSuccess) return FGATTN_ERR_CUDA;
+    if (d == 96) return launch_bwd_m<96>(prm, MQ, s);
     return d == 128 ? launch_bwd_m<128>(prm, MQ, s) : launch_bwd_m<64>(prm, MQ, s);
 }
 

@@ -175,7 +175,8 @@ fgattn_status fgattn_masked_forward(const void* q, const void* k, const void* v,
  *                            block keeps get zeros)
  *   delta               out  device fp32 [B][H][L]: workspace owned by the
  *                            caller; holds delta_i on return
- * Supported: d in {64, 128}, M in {16, 32, 64, 128} (a 128-row block runs as
+ * Supported: d in {64, 96, 128} (at d = 96 the products run on tiles padded
+ * with zero columns to 128), M in {16, 32, 64, 128} (a 128-row block runs as
  * two 64-row halves over its list), any N >= 1, any L >= 1.
  * P and ds are rounded to bf16 for the tensor-core products; accumulation in
  * fp32.  dk and dv are accumulated with float atomics (many query blocks keep

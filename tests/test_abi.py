@@ -166,8 +166,8 @@ def test_header_declares_backward():
     (dict(dk=P + 4), F.ERR_INVALID_ARG),
     (dict(delta=P + 2), F.ERR_INVALID_ARG),
     (dict(cap=63), F.ERR_CAPACITY),
-    (dict(d=96), F.ERR_UNSUPPORTED),
     (dict(d=80), F.ERR_UNSUPPORTED),
+    (dict(d=256), F.ERR_UNSUPPORTED),
     (dict(M=256), F.ERR_UNSUPPORTED),
     (dict(M=48), F.ERR_UNSUPPORTED),
 ])

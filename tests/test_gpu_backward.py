@@ -75,6 +75,8 @@ CASES = [
     # 128-row blocks (two 64-row halves over one list): ragged last block, a last block
     # whose second half is past L, one block
     (700, 128, 128, 16, 0.3, 1), (450, 64, 128, 5, 0.4, 2), (100, 128, 128, 64, 0.5, 1),
+    # d = 96 (tiles padded to 128 columns with zeros): every query-block height
+    (300, 96, 64, 16, 0.3, 2), (257, 96, 16, 1, 0.4, 1), (200, 96, 128, 5, 0.35, 1), (130, 96, 32, 4, 0.3, 1),
 ]
 
 
