@@ -33,8 +33,19 @@ def source_hash() -> str:
     return h.hexdigest()
 
 
+def _code_only(text: bytes) -> bytes:
+    """Source text without comments and trailing blanks: an edit to a comment does not
+    change the compiled kernel, so it does not change the kernel's hash."""
+    import re
+    t = text.decode()
+    t = re.sub(r"/\*.*?\*/", "", t, flags=re.S)
+    t = re.sub(r"//[^\n]*", "", t)
+    return "\n".join(line.rstrip() for line in t.splitlines() if line.strip()).encode()
+
+
 def kernel_hash(kernel: str) -> str:
-    """Hash of the sources one kernel is built from (ties a profile to a kernel version)."""
+    """Hash of the code (comments removed) of the sources one kernel is built from
+    (ties a profile to a kernel version)."""
     files = {"fwd": ["attention_fwd.cuh", "mask_row.cuh", "sm100_ptx.cuh"],
              "fwd_qm": ["attention_fwd.cuh", "attention_fwd_qm.cuh", "mask_row.cuh", "sm100_ptx.cuh"],
              "compact": ["compact_mask.cuh"],
@@ -42,7 +53,7 @@ def kernel_hash(kernel: str) -> str:
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(fh.read())
+            h.update(_code_only(fh.read()))
     return h.hexdigest()[:16]
 
 

@@ -7,7 +7,8 @@
 //     P^T  = exp(scale * K Q^T - lse)           dP^T = V dO^T
 //     dS^T = P^T o (dP^T - Delta),  Delta_i = dO_i . O_i
 //     dV  += P^T dO      dK += scale * dS^T Q    dQ^T += scale * K^T dS^T
-// per query block (b, h, qb) of MQ rows and each 128-key chunk of its list.
+// per work item -- MQ <= 64 query rows of block (b, h, qb); a 128-row block is
+// two items over the same list -- and each 128-key chunk of the list.
 //
 // Key-major, like the forward's kernel for short query blocks: a thread owns one
 // key of the chunk (TMEM lane), so P^T and dS^T go to TMEM as the A operands of
@@ -105,11 +106,11 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 
 struct alignas(64) BwdParams {
     CUtensorMap tmap_dk, tmap_dv;            // fp32 {D, L, B*H}, box {32, 16, 1}, 128B swizzle
-    const __nv_bfloat16 *q, *k, *v, *dout;  // [B][H][L][D]
+    const __nv_bfloat16 *q, *k, *v, *dout;  // [B][H][L][D], contiguous
     const float* lse;                        // [B][H][L], natural log (the forward's)
     const float* delta;                      // [B][H][L], dO_i . O_i
-    const int32_t* kept_idx;                 // [items][cap], or null: every key kept
-    const int32_t* kept_cnt;                 // [items]
+    const int32_t* kept_idx;                 // [B*H*QB][cap], or null: every key kept
+    const int32_t* kept_cnt;                 // [B*H*QB]
     float *dq, *dk, *dv;                     // fp32 [B][H][L][D]; dk and dv accumulate (zeroed first)
     int64_t cap, L;
     int64_t QB;      // query blocks of the lists (M rows each) per (b, h)
