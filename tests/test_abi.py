@@ -301,10 +301,3 @@ def test_tensors_on_another_device_are_refused(monkeypatch):
         F._require_current_device([("q", 0), ("k", 1)])
     with pytest.raises(ValueError, match="stream"):
         F._require_current_device([("stream", 2)])
-
-
-def test_autograd_module_refuses_host_tensors():
-    from fine_grained_sparse_fgattn_b200.autograd import tile_sparse_attention
-    q = torch.zeros((1, 1, 16, 64), dtype=torch.bfloat16)
-    with pytest.raises(ValueError):
-        tile_sparse_attention(q, q, q, None, None, 16, 16)

@@ -139,30 +139,3 @@ def test_backward_full_wan_layer(oracle):
     ref = oracle.backward(q0, k0, v0, g[:, :1], W.make_mask(w, 0, heads=h0), w.M, w.N, w.scale)
     got = tuple(t[:, :1].cpu().double().numpy() for t in (dq, dk, dv))
     print(compare_grads(got, ref))
-
-
-def test_autograd_function(oracle):
-    """tile_sparse_attention under torch.autograd: the same kernels as the two calls
-    (dq bit-identical; dk and dv sums of float reductions, equal up to their order),
-    and the gradients, cast to bf16 by autograd, still match the oracle."""
-    from fine_grained_sparse_fgattn_b200.autograd import tile_sparse_attention
-    L, d, M, N, H = 300, 128, 64, 16, 2
-    QB, G = -(-L // M), -(-L // N)
-    dev = torch.device("cuda", 0)
-    q, k, v = W.random_qkv(1, H, L, d, seed=21, std=1.5)
-    g = W.random_grad(1, H, L, d, seed=21)
-    mask = W.pack_tiles(W.random_tiles(1, H, QB, G, 0.3, seed=22))
-    idx, cnt = F.compact_mask(torch.from_numpy(mask.view(np.int32)).to(dev), 1, H, L, M, N)
-    qd, kd, vd = (t.to(dev).requires_grad_() for t in (q, k, v))
-    out = tile_sparse_attention(qd, kd, vd, idx, cnt, M, N)
-    out.backward(g.to(dev))
-    assert F.device_error() == 0
-    assert qd.grad.dtype == torch.bfloat16
-    out2, lse2 = F.forward(qd.detach(), kd.detach(), vd.detach(), idx, cnt, M, N)
-    assert torch.equal(out.detach(), out2)
-    dq, dk, dv = F.backward(qd.detach(), kd.detach(), vd.detach(), out2, g.to(dev), lse2, idx, cnt, M, N)
-    assert torch.equal(qd.grad, dq.to(torch.bfloat16))
-    for a, b in ((kd.grad, dk), (vd.grad, dv)):
-        assert (a.float() - b.to(torch.bfloat16).float()).abs().max().item() <= 1e-2 * b.abs().max().item()
-    ref = oracle.backward(q, k, v, g, mask, M, N, 1.0 / np.sqrt(d))
-    print(compare_grads(tuple(t.grad.cpu().double().numpy() for t in (qd, kd, vd)), ref))
