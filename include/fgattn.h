@@ -16,7 +16,9 @@
  *     asynchronously; argument validation happens synchronously on the host
  *     before anything is enqueued, and a call that returns an error status has
  *     enqueued nothing (fgattn_attention_from_host: unless the status is CUDA,
- *     which can leave the copies and kernels of earlier head groups enqueued).
+ *     which can leave the copies and kernels of earlier head groups enqueued;
+ *     fgattn_backward: unless the status is CUDA, which can leave the zeroing of
+ *     dk and dv and the delta pass enqueued).
  *   - Shapes: B batch, H heads, L tokens, d head dimension.
  *       QB = ceil(L / M) query blocks, G = ceil(L / N) key groups,
  *       W  = ceil(G / 32) mask words per query block.
