@@ -266,13 +266,17 @@ typedef struct {
     const uint32_t* mask;
     int64_t B, H, L, d, M, N;
     double scale;
-    double *dq, *dk, *dv;
-    int64_t first, last; /* this worker's share of heads */
+    int64_t bh;                /* the head */
+    int64_t row_first, row_last; /* this worker's query rows */
+    double *dq;                /* dq of the head (rows are disjoint between workers) */
+    double *dk, *dv;           /* this worker's partial sums over its rows, [L][d] */
     int status;
 } bjob_t;
 
-static int backward_head(const bjob_t* J, int64_t bh) {
-    const int64_t L = J->L, d = J->d, M = J->M, N = J->N;
+/* Rows row_first .. row_last-1 of one head: dq of those rows, and their terms
+ * of dk and dv added into the worker's own partial sums. */
+static int backward_rows(const bjob_t* J) {
+    const int64_t L = J->L, d = J->d, M = J->M, N = J->N, bh = J->bh;
     const int64_t QB = (L + M - 1) / M;
     const int64_t G = (L + N - 1) / N;
     const int64_t W = (G + 31) / 32;
@@ -280,15 +284,15 @@ static int backward_head(const bjob_t* J, int64_t bh) {
     const uint16_t* K = J->k + bh * L * d;
     const uint16_t* V = J->v + bh * L * d;
     const uint16_t* DO = J->dout + bh * L * d;
-    double* dq = J->dq + bh * L * d;
-    double* dk = J->dk + bh * L * d;
-    double* dv = J->dv + bh * L * d;
+    double* dq = J->dq;
+    double* dk = J->dk;
+    double* dv = J->dv;
     double* s = (double*)malloc((size_t)L * sizeof(double));
     double* dp = (double*)malloc((size_t)L * sizeof(double));
     char* kept = (char*)malloc((size_t)G);
     if (!s || !dp || !kept) { free(s); free(dp); free(kept); return -2; }
     for (int64_t x = 0; x < L * d; ++x) { dk[x] = 0.0; dv[x] = 0.0; }
-    for (int64_t i = 0; i < L; ++i) {
+    for (int64_t i = J->row_first; i < J->row_last; ++i) {
         const int64_t qb = i / M;
         const uint32_t* mrow = J->mask + (bh * QB + qb) * W;
         for (int64_t g = 0; g < G; ++g) kept[g] = (char)tile_kept(mrow, qb, g, L, M, N);
@@ -353,45 +357,60 @@ static int backward_head(const bjob_t* J, int64_t bh) {
 
 static void* bworker(void* arg) {
     bjob_t* J = (bjob_t*)arg;
-    for (int64_t bh = J->first; bh < J->last; ++bh) {
-        int st = backward_head(J, bh);
-        if (st) { J->status = st; break; }
-    }
+    J->status = backward_rows(J);
     return NULL;
 }
 
-/* Gradients dq, dk, dv of every head (see above).  Returns 0 on success. */
+/* Gradients dq, dk, dv of every head (see above).  Returns 0 on success.
+ * Heads one after the other; the rows of a head split between up to nthreads
+ * workers, each summing its rows' terms of dk and dv on its own; the head's dk
+ * and dv are then those partial sums added in worker order. */
 int oracle_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
                               const uint32_t* mask, int64_t B, int64_t H, int64_t L, int64_t d, int64_t M,
                               int64_t N, double scale, double* dq, double* dk, double* dv, int nthreads) {
-    const int64_t heads = B * H;
     if (nthreads < 1) nthreads = 1;
-    if (nthreads > heads) nthreads = (int)(heads > 0 ? heads : 1);
+    if (nthreads > L) nthreads = (int)L;
+    /* partial sums take 2 * L * d doubles per worker: at most about 1 GiB of them */
+    const int64_t per = 2 * L * d * (int64_t)sizeof(double);
+    const int64_t cap = per > 0 ? (((int64_t)1 << 30) / per) : 1;
+    if (cap < nthreads) nthreads = cap < 1 ? 1 : (int)cap;
     bjob_t* jobs = (bjob_t*)calloc((size_t)nthreads, sizeof(bjob_t));
     pthread_t* tid = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
-    if (!jobs || !tid) { free(jobs); free(tid); return -2; }
-    for (int w = 0; w < nthreads; ++w) {
-        bjob_t* J = &jobs[w];
-        J->q = q; J->k = k; J->v = v; J->dout = dout; J->mask = mask;
-        J->B = B; J->H = H; J->L = L; J->d = d; J->M = M; J->N = N; J->scale = scale;
-        J->dq = dq; J->dk = dk; J->dv = dv;
-        J->first = heads * w / nthreads;
-        J->last = heads * (w + 1) / nthreads;
-        J->status = 0;
-    }
+    double* part = (double*)malloc((size_t)nthreads * (size_t)per);
+    if (!jobs || !tid || !part) { free(jobs); free(tid); free(part); return -2; }
     int status = 0;
-    if (nthreads == 1) {
-        bworker(&jobs[0]);
-        status = jobs[0].status;
-    } else {
-        int started = 0;
+    for (int64_t bh = 0; bh < B * H && !status; ++bh) {
         for (int w = 0; w < nthreads; ++w) {
-            if (pthread_create(&tid[w], NULL, bworker, &jobs[w]) != 0) { status = -3; break; }
-            ++started;
+            bjob_t* J = &jobs[w];
+            J->q = q; J->k = k; J->v = v; J->dout = dout; J->mask = mask;
+            J->B = B; J->H = H; J->L = L; J->d = d; J->M = M; J->N = N; J->scale = scale;
+            J->bh = bh;
+            J->row_first = L * w / nthreads;
+            J->row_last = L * (w + 1) / nthreads;
+            J->dq = dq + bh * L * d;
+            J->dk = part + (size_t)w * 2 * (size_t)(L * d);
+            J->dv = J->dk + L * d;
+            J->status = 0;
         }
-        for (int w = 0; w < started; ++w) pthread_join(tid[w], NULL);
+        if (nthreads == 1) {
+            bworker(&jobs[0]);
+        } else {
+            int started = 0;
+            for (int w = 0; w < nthreads; ++w) {
+                if (pthread_create(&tid[w], NULL, bworker, &jobs[w]) != 0) { status = -3; break; }
+                ++started;
+            }
+            for (int w = 0; w < started; ++w) pthread_join(tid[w], NULL);
+        }
         for (int w = 0; w < nthreads && !status; ++w) status = jobs[w].status;
+        if (status) break;
+        double* hk = dk + bh * L * d;
+        double* hv = dv + bh * L * d;
+        for (int64_t x = 0; x < L * d; ++x) { hk[x] = 0.0; hv[x] = 0.0; }
+        for (int w = 0; w < nthreads; ++w)
+            for (int64_t x = 0; x < L * d; ++x) { hk[x] += jobs[w].dk[x]; hv[x] += jobs[w].dv[x]; }
     }
+    free(part);
     free(jobs);
     free(tid);
     return status;
