@@ -75,3 +75,16 @@ def test_granularity_sweep_targets(N):
     assert abs(W.score_sparsity(tiles, w) - w.sparsity) < 1e-3
     i = np.arange(w.L)
     assert tiles[:, :, i // w.M, i // w.N].all()
+
+
+def test_random_grad_is_seeded_and_independent_of_qkv():
+    """The upstream gradient of the backward cases: same seed, same values; another
+    seed, other values; and not a copy of the q/k/v streams of the same seed."""
+    a = W.random_grad(1, 2, 40, 16, seed=5)
+    b = W.random_grad(1, 2, 40, 16, seed=5)
+    c = W.random_grad(1, 2, 40, 16, seed=6)
+    q, k, v = W.random_qkv(1, 2, 40, 16, seed=5)
+    assert a.dtype == torch.bfloat16 and a.shape == (1, 2, 40, 16)
+    assert torch.equal(a, b) and not torch.equal(a, c)
+    assert not any(torch.equal(a, t) for t in (q, k, v))
+    assert abs(a.float().std().item() - 1.0) < 0.2
